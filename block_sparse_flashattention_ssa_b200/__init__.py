@@ -1,0 +1,198 @@
+"""BLASST skip-softmax attention for B200 (sm_100a): Python binding.
+
+Argument marshalling over the C ABI declared in ``include/ssa.h`` and
+implemented in ``libssa.so`` (built in-tree by ``build.py``). Every step of
+the computation runs in the library's CUDA kernels; torch only provides
+device memory and streams. There is no CPU fallback: importing this package
+fails loudly when the library is missing.
+
+Entry points (same names as the C ABI, without the ``ssa_`` prefix):
+  fwd          skip-softmax attention forward (optionally with per-tile
+               diagnostics, the ``ssa_fwd_ex`` call)
+  calibrate    dense attention + skip counts at N thresholds at once
+  resolve      threshold_scale_factor = a * exp(b * target_sparsity)
+  fit_logspace log-space least-squares fit of (a, b)
+  num_qblocks  number of 128-row query blocks of a batch
+  get_error    synchronise and read/clear the device status word
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_PKG, "libssa.so")
+TILE = 128
+MAX_THRESHOLDS = 32
+
+SSA_OK = 0
+SSA_ERR_INVALID_ARG = -1
+SSA_ERR_UNSUPPORTED = -2
+SSA_ERR_CUDA = -3
+SSA_ERR_TIMEOUT = -4
+SSA_ERR_DEVICE_ARG = -5
+
+
+class SSAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status} ({_lib.ssa_status_string(status).decode()})")
+
+
+def _load():
+    if not os.path.exists(_SO):
+        raise ImportError(f"libssa.so is not built ({_SO}); run block_sparse_flashattention_ssa_b200/build.py")
+    L = ctypes.CDLL(_SO)
+    vp, i32, f32, f64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_double
+    L.ssa_fwd.restype = i32
+    L.ssa_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp]
+    L.ssa_fwd_ex.restype = i32
+    L.ssa_fwd_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp, vp, vp]
+    L.ssa_calibrate.restype = i32
+    L.ssa_calibrate.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32, vp, vp, vp]
+    L.ssa_resolve.restype = f64
+    L.ssa_resolve.argtypes = [f64, f64, f64]
+    L.ssa_fit_logspace.restype = i32
+    L.ssa_fit_logspace.argtypes = [vp, vp, i32, vp, vp, vp, vp]
+    L.ssa_num_qblocks.restype = i32
+    L.ssa_num_qblocks.argtypes = [vp, i32]
+    L.ssa_get_error.restype = i32
+    L.ssa_get_error.argtypes = [vp]
+    L.ssa_status_string.restype = ctypes.c_char_p
+    L.ssa_status_string.argtypes = [i32]
+    return L
+
+
+_lib = _load()
+
+
+def lib():
+    """The loaded ctypes library (for callers that marshal raw pointers)."""
+    return _lib
+
+
+def library_path() -> str:
+    return _SO
+
+
+def _check(rc: int, what: str):
+    if rc != SSA_OK:
+        raise SSAError(rc, what)
+
+
+def _stream_handle(stream):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _shape(q):
+    if q.dim() != 3:
+        raise ValueError("q, k, v must be [total_tokens, H, D]")
+    return q.shape[0], q.shape[1], q.shape[2]
+
+
+def num_qblocks(cu_seqlens) -> int:
+    """Total 128-row query blocks over the batch (from a host copy of cu_seqlens)."""
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens if not hasattr(cu_seqlens, "cpu") else cu_seqlens.cpu()),
+                              dtype=np.int32)
+    n = _lib.ssa_num_qblocks(cu.ctypes.data, len(cu) - 1)
+    if n < 0:
+        raise SSAError(n, "ssa_num_qblocks")
+    return n
+
+
+def fwd(q, k, v, cu_seqlens, max_seqlen: int, threshold_scale_factor: float = 0.0, softmax_scale: float = 0.0,
+        out=None, skip_counter=None, decision_bitmap=None, tile_stat=None, stream=None):
+    """Skip-softmax attention forward. q, k, v: CUDA bf16 [total_tokens, H, D];
+    cu_seqlens: CUDA int32 [B+1]. Returns ``out`` (allocated when None).
+    ``skip_counter`` (int32 [H, Q]), ``decision_bitmap`` (int32/uint32
+    [H, Q, ceil(T/32)]) and ``tile_stat`` (float32 [H, Q, T]) are optional
+    caller-allocated outputs; passing either of the last two selects the
+    diagnostic call ``ssa_fwd_ex``."""
+    import torch
+
+    total, H, D = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    batch = cu_seqlens.numel() - 1
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D,
+            float(softmax_scale), float(threshold_scale_factor), _ptr(out), _ptr(skip_counter)]
+    if decision_bitmap is not None or tile_stat is not None:
+        rc = _lib.ssa_fwd_ex(*args, _ptr(decision_bitmap), _ptr(tile_stat), _stream_handle(stream))
+        _check(rc, "ssa_fwd_ex")
+    else:
+        _check(_lib.ssa_fwd(*args, _stream_handle(stream)), "ssa_fwd")
+    return out
+
+
+def calibrate(q, k, v, cu_seqlens, max_seqlen: int, thresholds, softmax_scale: float = 0.0, out=None, counts=None,
+              stream=None):
+    """Dense attention plus, per (head, q-block) unit, the number of KV tiles
+    that would be skipped at each raw lambda in ``thresholds``. Returns
+    (out, counts[H, Q, N])."""
+    import torch
+
+    total, H, D = _shape(q)
+    th = np.ascontiguousarray(thresholds, dtype=np.float32)
+    if out is None:
+        out = torch.empty_like(q)
+    if counts is None:
+        Q = num_qblocks(cu_seqlens)
+        counts = torch.empty((H, Q, len(th)), dtype=torch.int32, device=q.device)
+    batch = cu_seqlens.numel() - 1
+    rc = _lib.ssa_calibrate(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D,
+                            float(softmax_scale), th.ctypes.data, len(th), _ptr(out), _ptr(counts),
+                            _stream_handle(stream))
+    _check(rc, "ssa_calibrate")
+    return out, counts
+
+
+def resolve(a: float, b: float, target_sparsity: float) -> float:
+    return float(_lib.ssa_resolve(a, b, target_sparsity))
+
+
+def fit_logspace(sparsity, scale_factor):
+    """Returns (a, b, s_min, s_max)."""
+    s = np.ascontiguousarray(sparsity, dtype=np.float64)
+    sf = np.ascontiguousarray(scale_factor, dtype=np.float64)
+    if s.shape != sf.shape:
+        raise ValueError("sparsity and scale_factor differ in length")
+    out = [ctypes.c_double() for _ in range(4)]
+    _check(_lib.ssa_fit_logspace(s.ctypes.data, sf.ctypes.data, len(s), *[ctypes.byref(o) for o in out]),
+           "ssa_fit_logspace")
+    return tuple(o.value for o in out)
+
+
+def get_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status."""
+    return int(_lib.ssa_get_error(_stream_handle(stream)))
+
+
+def check_device(stream=None):
+    """Raise SSAError when a kernel recorded an error on this device."""
+    _check(get_error(stream), "device status")
+
+
+def max_tiles(max_seqlen: int) -> int:
+    return (int(max_seqlen) + TILE - 1) // TILE
+
+
+def bitmap_words(max_seqlen: int) -> int:
+    return (max_tiles(max_seqlen) + 31) // 32
+
+
+def threshold_log2(threshold_scale_factor: float, s_kv: int) -> float:
+    """Host helper for callers and reports: log2(tsf / S_kv), -inf when tsf <= 0."""
+    if threshold_scale_factor <= 0:
+        return -math.inf
+    return math.log2(threshold_scale_factor / s_kv)

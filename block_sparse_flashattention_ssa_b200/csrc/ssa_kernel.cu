@@ -1,0 +1,655 @@
+// BLASST skip-softmax attention for B200 (sm_100a): forward with tile
+// skipping and the multi-threshold calibration pass.
+//
+// One CTA walks the KV tiles of one 128-row query block of one (sequence,
+// head). Warp roles:
+//   warp 4  TMA producer: Q once, K tiles through a 3-stage ring, and V tiles
+//           through a 2-stage ring -- V of tile j only once the softmax warps
+//           have decided to keep tile j (skipped tiles issue no V load);
+//   warp 5  tcgen05 issuer: S_j = Q K_j^T into one of two TMEM S buffers
+//           (issued one tile ahead), and O += P_j V_j from a TMEM copy of P_j
+//           (kept tiles only);
+//   warps 0-3  softmax, one query row per thread: row max of S_j in the log2
+//           domain, the CTA-wide skip vote d_j < log2(lambda) (Model-Optimizer
+//           commit page, "Triton kernels": tiles whose max score is far below
+//           the running max are skipped, no V load, softmax or accumulation),
+//           exponentials with a lazily rescaled reference max, P to TMEM, and
+//           the epilogue O / l -> bf16.
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O [256,256+D) P0 [384,448)
+// P1 [448,512), P stored as packed bf16 pairs.
+//
+// Every wait on an mbarrier is bounded in time; when one runs out the CTA
+// records SSA_ERR_TIMEOUT in the device status word, the other roles see the
+// abort flag at their next wait, in-flight TMA loads and MMAs are drained
+// (again with a bound) and TMEM is released before the CTA exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "sm100.cuh"
+#include "ssa.h"
+
+namespace ssa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBM = SSA_TILE;  // query rows per tile
+constexpr int kBN = SSA_TILE;  // key/value rows per tile
+constexpr int kThreads = 192;
+constexpr int kTmaWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
+constexpr int kDecRing = 4;  // > kKStages - 1: bounds how far the vote runs ahead of the V producer
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 256 before a rescale
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr int kStatusTimeout = 1;
+constexpr int kStatusDeviceArg = 2;
+constexpr uint32_t kFull = 0xFFFFFFFFu;
+
+enum Mode : int { kDense = 0, kSkip = 1, kCalib = 2 };
+
+__device__ int g_status;  // sticky error bits of this device, read by ssa_get_error
+
+struct Params {
+  const int32_t* cu_seqlens;
+  __nv_bfloat16* out;
+  int32_t* skip_counter;
+  int32_t* counts;
+  uint32_t* bitmap;
+  float* tile_stat;
+  int batch, total_tokens, num_heads, max_tiles, bitmap_words;
+  float c;    // fp32(softmax_scale * log2 e)
+  float tsf;  // threshold_scale_factor (kSkip)
+  int n_cal;
+  float Lcal[SSA_MAX_THRESHOLDS];  // fp32(log2 lambda_k) (kCalib)
+};
+
+struct Ctl {
+  uint64_t bar_q;
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], s_free[2], p_ready[2], pv_done[2];
+  uint64_t dec_ready[kDecRing], red_bar[2], drain;
+  uint32_t tmem_base;
+  int abort_flag;
+  int dec[kDecRing];
+  float red[2][4];
+  int seq, qb, S, start, gqb, nq_total;
+};
+
+template <int D>
+struct Layout {
+  static constexpr int kTileBytes = kBM * D * 2;  // 128 rows x D bf16, as D/64 chunks of 128 rows x 128 B
+  static constexpr int kChunkBytes = kBM * 128;
+  static constexpr int kQ = 0;
+  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kV = kK + kKStages * kTileBytes;
+  static constexpr int kCtl = kV + kVStages * kTileBytes;
+  static constexpr int kBytes = kCtl + static_cast<int>(sizeof(Ctl));
+  static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B (128B swizzle atoms)
+};
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicOr(&g_status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// Warp-uniform bounded wait: every lane returns the same verdict.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  return __all_sync(kFull, wait_bar(bar, parity, abort_flag));
+}
+
+// Wait that ignores the abort flag (used to drain in-flight async work).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_status, kStatusTimeout);
+      return;
+    }
+  }
+}
+
+template <int D, int MODE, bool EX>
+__global__ void __launch_bounds__(kThreads, 1)
+    ssa_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params p) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl& ctl = *reinterpret_cast<Ctl*>(smem + L::kCtl);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int head = blockIdx.y;
+
+  // Locate this CTA's (sequence, q-block) and validate cu_seqlens.
+  if (threadIdx.x == 0) {
+    int acc = 0, seq = -1, qb = 0, start = 0, S = 0, gqb = 0, bad = 0;
+    int prev = p.cu_seqlens[0];
+    if (prev < 0) bad = 1;
+    for (int b = 0; b < p.batch && !bad; ++b) {
+      const int nxt = p.cu_seqlens[b + 1];
+      const int len = nxt - prev;
+      if (len < 0 || nxt > p.total_tokens) {
+        bad = 1;
+        break;
+      }
+      const int nq = (len + kBM - 1) / kBM;
+      if (seq < 0 && static_cast<int>(blockIdx.x) < acc + nq) {
+        seq = b;
+        qb = blockIdx.x - acc;
+        gqb = blockIdx.x;
+        start = prev;
+        S = len;
+      }
+      acc += nq;
+      prev = nxt;
+    }
+    if (!bad && seq >= 0 && (EX && (S + kBN - 1) / kBN > p.max_tiles)) bad = 1;
+    if (bad) {
+      if (blockIdx.x == 0) atomicOr(&g_status, kStatusDeviceArg);
+      seq = -1;
+    }
+    ctl.seq = seq;
+    ctl.qb = qb;
+    ctl.S = S;
+    ctl.start = start;
+    ctl.gqb = gqb;
+    ctl.nq_total = acc;
+  }
+  __syncthreads();
+  if (ctl.seq < 0) return;  // uniform: no unit for this CTA (or bad input)
+
+  const int qb = ctl.qb, S = ctl.S, seq_start = ctl.start;
+  const int nkv = (S + kBN - 1) / kBN;
+  const int64_t unit = static_cast<int64_t>(head) * ctl.nq_total + ctl.gqb;
+  volatile int* abort_flag = &ctl.abort_flag;
+
+  const uint32_t bar_q = smem_u32(&ctl.bar_q);
+  auto k_full = [&](int i) { return smem_u32(&ctl.k_full[i]); };
+  auto k_empty = [&](int i) { return smem_u32(&ctl.k_empty[i]); };
+  auto v_full = [&](int i) { return smem_u32(&ctl.v_full[i]); };
+  auto v_empty = [&](int i) { return smem_u32(&ctl.v_empty[i]); };
+  auto s_full = [&](int i) { return smem_u32(&ctl.s_full[i]); };
+  auto s_free = [&](int i) { return smem_u32(&ctl.s_free[i]); };
+  auto p_ready = [&](int i) { return smem_u32(&ctl.p_ready[i]); };
+  auto pv_done = [&](int i) { return smem_u32(&ctl.pv_done[i]); };
+  auto dec_ready = [&](int i) { return smem_u32(&ctl.dec_ready[i]); };
+  auto red_bar = [&](int i) { return smem_u32(&ctl.red_bar[i]); };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(k_full(i), 1);
+      mbar_init(k_empty(i), 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(v_full(i), 1);
+      mbar_init(v_empty(i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full(i), 1);
+      mbar_init(s_free(i), 128);
+      mbar_init(p_ready(i), 128);
+      mbar_init(pv_done(i), 1);
+      mbar_init(red_bar(i), 4);
+    }
+    for (int i = 0; i < kDecRing; ++i) mbar_init(dec_ready(i), 1);
+    mbar_init(smem_u32(&ctl.drain), 1);
+    ctl.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(&ctl.tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = ctl.tmem_base;
+
+  if (warp == kTmaWarp) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const uint32_t q_s = smem_u32(smem + L::kQ);
+      mbar_arrive_expect_tx(bar_q, L::kTileBytes);
+      for (int ch = 0; ch < D / 64; ++ch) tma_load_3d(q_s + ch * L::kChunkBytes, &tmQ, bar_q, ch * 64, head, seq_start + qb * kBM);
+      int k_issued = 0, v_issued = 0;
+      bool ok = true;
+      for (int j = 0; j < nkv && ok; ++j) {
+        for (; k_issued < nkv && k_issued < j + kKStages; ++k_issued) {
+          const int st = k_issued % kKStages;
+          if (k_issued >= kKStages && !wait_bar(k_empty(st), ((k_issued / kKStages) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = smem_u32(smem + L::kK + st * L::kTileBytes);
+          mbar_arrive_expect_tx(k_full(st), L::kTileBytes);
+          for (int ch = 0; ch < D / 64; ++ch)
+            tma_load_3d(dst + ch * L::kChunkBytes, &tmK, k_full(st), ch * 64, head, seq_start + k_issued * kBN);
+        }
+        if (!ok) break;
+        bool skip = false;
+        if (MODE == kSkip) {
+          if (!wait_bar(dec_ready(j % kDecRing), (j / kDecRing) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          skip = reinterpret_cast<volatile int*>(ctl.dec)[j % kDecRing] != 0;
+        }
+        if (!skip) {
+          const int vs = v_issued % kVStages;
+          if (v_issued >= kVStages && !wait_bar(v_empty(vs), ((v_issued / kVStages) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = smem_u32(smem + L::kV + vs * L::kTileBytes);
+          mbar_arrive_expect_tx(v_full(vs), L::kTileBytes);
+          for (int ch = 0; ch < D / 64; ++ch)
+            tma_load_3d(dst + ch * L::kChunkBytes, &tmV, v_full(vs), ch * 64, head, seq_start + j * kBN);
+          ++v_issued;
+        }
+      }
+      if (!ok) {  // drain the loads still in flight before shared memory goes away
+        drain_wait(bar_q, 0);
+        for (int st = 0; st < kKStages; ++st)
+          if (k_issued > st) drain_wait(k_full(st), ((k_issued - 1 - st) / kKStages) & 1);
+        for (int st = 0; st < kVStages; ++st)
+          if (v_issued > st) drain_wait(v_full(st), ((v_issued - 1 - st) / kVStages) & 1);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------- tcgen05 issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
+      const uint32_t q_s = smem_u32(smem + L::kQ);
+      auto issue_qk = [&](int t) -> bool {
+        const int st = t % kKStages;
+        if (!wait_bar(k_full(st), (t / kKStages) & 1, abort_flag)) return false;
+        const int sb = t & 1;
+        if (t >= 2 && !wait_bar(s_free(sb), ((t >> 1) - 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t k_s = smem_u32(smem + L::kK + st * L::kTileBytes);
+        const uint32_t d_tmem = tmem + (sb ? kColS1 : kColS0);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          // K-major, 128B swizzle: 16-element k slices are 32 B apart inside a
+          // 128-B row; every 64 elements start a new 16 KB chunk.
+          const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
+          mma_ss(d_tmem, smem_desc_sw128(q_s + off, 16, 1024), smem_desc_sw128(k_s + off, 16, 1024), idesc_qk,
+                 ks > 0 ? 1u : 0u);
+        }
+        tc_commit(s_full(sb));
+        tc_commit(k_empty(st));
+        return true;
+      };
+      bool ok = wait_bar(bar_q, 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        ok = issue_qk(0);
+      }
+      int kept = 0;
+      for (int j = 0; ok && j < nkv; ++j) {
+        if (j + 1 < nkv && !(ok = issue_qk(j + 1))) break;
+        if (!(ok = wait_bar(p_ready(j & 1), (j >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        const bool skip = (MODE == kSkip) && reinterpret_cast<volatile int*>(ctl.dec)[j % kDecRing] != 0;
+        if (skip) continue;
+        const int vs = kept % kVStages;
+        if (!(ok = wait_bar(v_full(vs), (kept / kVStages) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t p_tmem = tmem + ((kept & 1) ? kColP1 : kColP0);
+        const uint32_t v_s = smem_u32(smem + L::kV + vs * L::kTileBytes);
+#pragma unroll
+        for (int ks = 0; ks < kBN / 16; ++ks) {
+          // V is MN-major (d contiguous): 16 kv rows = 2 KB per k step; the
+          // second 64-column chunk of d sits one 16 KB chunk further (LBO).
+          mma_ts(tmem + kColO, p_tmem + ks * 8, smem_desc_sw128(v_s + ks * 16 * 128, L::kChunkBytes, 1024),
+                 idesc_pv, (kept > 0 || ks > 0) ? 1u : 0u);
+        }
+        tc_commit(v_empty(vs));
+        tc_commit(pv_done(kept & 1));
+        ++kept;
+      }
+      if (!ok) {  // let every MMA issued so far finish before TMEM is released
+        tc_commit(smem_u32(&ctl.drain));
+        drain_wait(smem_u32(&ctl.drain), 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int row = warp * 32 + lane;
+    const bool row_valid = qb * kBM + row < S;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const float c = p.c;
+    float Lthr = -INFINITY;
+    if (MODE == kSkip) Lthr = static_cast<float>(log2(static_cast<double>(p.tsf) / static_cast<double>(S)));
+    float m_true = -INFINITY;  // running max of kept tiles (the skip rule's m_r)
+    float m_used = -INFINITY;  // reference max of the exponentials (lags m_true by < kRescaleThreshold)
+    float l = 0.f;
+    int kept = 0, nskip = 0;
+    int cnt[SSA_MAX_THRESHOLDS];
+#pragma unroll
+    for (int k = 0; k < SSA_MAX_THRESHOLDS; ++k) cnt[k] = 0;
+    uint32_t bits = 0;
+    bool ok = true;
+
+    for (int j = 0; j < nkv; ++j) {
+      const int sb = j & 1;
+      if (!(ok = warp_wait(s_full(sb), (j >> 1) & 1, abort_flag))) break;
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld_x128(lane_base + (sb ? kColS1 : kColS0), sr);
+      tc_fence_before();
+      mbar_arrive(s_free(sb));
+      float s[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
+      const int valid = S - j * kBN;
+      if (valid < kBN) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i >= valid) s[i] = -INFINITY;
+      }
+      float mx[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+      for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], s[i]);
+      const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                         c;
+
+      bool skip = false;
+      if (MODE != kDense || EX) {
+        float dr = row_valid ? (tmax - m_true) : -INFINITY;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dr = fmaxf(dr, __shfl_xor_sync(kFull, dr, o));
+        if (lane == 0) {
+          ctl.red[sb][warp] = dr;
+          mbar_arrive(red_bar(sb));
+        }
+        if (!(ok = warp_wait(red_bar(sb), (j >> 1) & 1, abort_flag))) break;
+        volatile float* red = ctl.red[sb];
+        const float d = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+        if (MODE == kSkip) skip = d < Lthr;
+        if (MODE == kCalib) {
+#pragma unroll
+          for (int k = 0; k < SSA_MAX_THRESHOLDS; ++k) cnt[k] += (k < p.n_cal && d < p.Lcal[k]) ? 1 : 0;
+        }
+        if (EX && threadIdx.x == 0) {
+          if (p.tile_stat) p.tile_stat[unit * p.max_tiles + j] = d;
+          bits |= (skip ? 1u : 0u) << (j & 31);
+          if ((j & 31) == 31 || j == nkv - 1) {
+            if (p.bitmap) p.bitmap[unit * p.bitmap_words + (j >> 5)] = bits;
+            bits = 0;
+          }
+        }
+        if (MODE == kSkip && threadIdx.x == 0) {
+          reinterpret_cast<volatile int*>(ctl.dec)[j % kDecRing] = skip ? 1 : 0;
+          mbar_arrive(dec_ready(j % kDecRing));
+        }
+      }
+      if (skip) {
+        ++nskip;
+        mbar_arrive(p_ready(sb));
+        continue;
+      }
+
+      // Kept tile: online softmax update.
+      const float m_new = fmaxf(m_true, tmax);
+      m_true = m_new;
+      float alpha = 1.f;
+      if (__any_sync(kFull, m_new > m_used + kRescaleThreshold)) {
+        alpha = ex2_approx(m_used - m_new);  // 0 before the first kept tile
+        m_used = m_new;
+        if (kept > 0) {
+          if (!(ok = warp_wait(pv_done((kept - 1) & 1), ((kept - 1) >> 1) & 1, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t o[32];
+            tmem_ld_x32(lane_base + kColO + ch * 32, o);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st_x32(lane_base + kColO + ch * 32, o);
+          }
+        }
+      }
+      l *= alpha;
+      const float neg_m = -m_used;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = ex2_approx(fmaf(s[2 * i], c, neg_m));
+        const float p1 = ex2_approx(fmaf(s[2 * i + 1], c, neg_m));
+        rs[i & 3] += p0 + p1;
+        pk[i] = pack_bf16x2(p0, p1);
+      }
+      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      if (kept >= 2 && !(ok = warp_wait(pv_done(kept & 1), ((kept - 2) >> 1) & 1, abort_flag))) break;
+      tmem_st_x64(lane_base + ((kept & 1) ? kColP1 : kColP0), pk);
+      tc_fence_before();
+      mbar_arrive(p_ready(sb));
+      ++kept;
+    }
+
+    // Epilogue: O / l -> bf16, masked row stores; per-unit counters.
+    if (ok && kept > 0) ok = warp_wait(pv_done((kept - 1) & 1), ((kept - 1) >> 1) & 1, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      __nv_bfloat16* orow =
+          p.out + (static_cast<int64_t>(seq_start + qb * kBM + row) * p.num_heads + head) * static_cast<int64_t>(D);
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t o[32];
+        tmem_ld_x32(lane_base + kColO + ch * 32, o);
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+      if (threadIdx.x == 0) {
+        if (p.skip_counter) p.skip_counter[unit] = nskip;
+        if (MODE == kCalib) {
+#pragma unroll
+          for (int k = 0; k < SSA_MAX_THRESHOLDS; ++k)
+            if (k < p.n_cal) p.counts[unit * p.n_cal + k] = cnt[k];
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [total_tokens, H, D] bf16 viewed as a 3-D tensor (d, head, token); box of
+// 64 d x 1 head x 128 tokens with 128-byte swizzle. Rows past total_tokens
+// read as zero.
+bool make_tensor_map(CUtensorMap* map, const void* base, int total_tokens, int H, int D) {
+  auto encode = encode_fn();
+  if (!encode) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(total_tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kBN)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct Call {
+  const void *q, *k, *v;
+  const int32_t* cu;
+  int batch, total_tokens, max_seqlen, H, D;
+  float softmax_scale;
+  void* out;
+  cudaStream_t stream;
+};
+
+// Host-side argument check. total_tokens == 0 is a valid no-op whatever the
+// data pointers are (an empty batch has no storage).
+int validate(const Call& a) {
+  if (!a.cu || a.batch < 1 || a.total_tokens < 0 || a.max_seqlen < 0 || a.H < 1 || a.H > 65535)
+    return SSA_ERR_INVALID_ARG;
+  if (std::isnan(a.softmax_scale) || std::isinf(a.softmax_scale)) return SSA_ERR_INVALID_ARG;
+  if (a.D != 64 && a.D != 128) return SSA_ERR_UNSUPPORTED;
+  if (a.total_tokens == 0) return SSA_OK;
+  if (!a.q || !a.k || !a.v || !a.out) return SSA_ERR_INVALID_ARG;
+  for (const void* ptr : {a.q, a.k, a.v, static_cast<const void*>(a.out)})
+    if (reinterpret_cast<uintptr_t>(ptr) & 15u) return SSA_ERR_UNSUPPORTED;
+  return SSA_OK;
+}
+
+Params base_params(const Call& a) {
+  Params p{};
+  p.cu_seqlens = a.cu;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.batch = a.batch;
+  p.total_tokens = a.total_tokens;
+  p.num_heads = a.H;
+  p.max_tiles = (a.max_seqlen + kBN - 1) / kBN;
+  p.bitmap_words = (p.max_tiles + 31) / 32;
+  const double scale = a.softmax_scale > 0.f ? static_cast<double>(a.softmax_scale) : 1.0 / std::sqrt(static_cast<double>(a.D));
+  p.c = static_cast<float>(scale * 1.4426950408889634073599246810019);
+  return p;
+}
+
+template <int D, int MODE, bool EX>
+int launch(const Call& a, const Params& p) {
+  CUtensorMap tq, tk, tv;
+  if (!make_tensor_map(&tq, a.q, a.total_tokens, a.H, D) || !make_tensor_map(&tk, a.k, a.total_tokens, a.H, D) ||
+      !make_tensor_map(&tv, a.v, a.total_tokens, a.H, D))
+    return SSA_ERR_CUDA;
+  auto kernel = ssa_attention_kernel<D, MODE, EX>;
+  constexpr int smem = Layout<D>::kAlloc;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return SSA_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>((a.total_tokens + kBM - 1) / kBM + a.batch), static_cast<unsigned>(a.H));
+  kernel<<<grid, kThreads, smem, a.stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+}
+
+template <int MODE, bool EX>
+int dispatch_d(const Call& a, const Params& p) {
+  return a.D == 64 ? launch<64, MODE, EX>(a, p) : launch<128, MODE, EX>(a, p);
+}
+
+int fwd_impl(const Call& a, float tsf, int32_t* skip_counter, uint32_t* bitmap, float* tile_stat) {
+  int rc = validate(a);
+  if (rc != SSA_OK) return rc;
+  if (std::isnan(tsf) || std::isinf(tsf)) return SSA_ERR_INVALID_ARG;
+  if ((bitmap || tile_stat) && a.max_seqlen < 1) return SSA_ERR_INVALID_ARG;
+  if (a.total_tokens == 0) return SSA_OK;
+  Params p = base_params(a);
+  p.skip_counter = skip_counter;
+  p.bitmap = bitmap;
+  p.tile_stat = tile_stat;
+  p.tsf = tsf;
+  const bool ex = bitmap || tile_stat;
+  if (tsf > 0.f) return ex ? dispatch_d<kSkip, true>(a, p) : dispatch_d<kSkip, false>(a, p);
+  return ex ? dispatch_d<kDense, true>(a, p) : dispatch_d<kDense, false>(a, p);
+}
+
+}  // namespace
+}  // namespace ssa
+
+using namespace ssa;
+
+extern "C" int ssa_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                       int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                       float threshold_scale_factor, void* out, int32_t* skip_counter, void* stream) {
+  const Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
+               static_cast<cudaStream_t>(stream)};
+  return fwd_impl(a, threshold_scale_factor, skip_counter, nullptr, nullptr);
+}
+
+extern "C" int ssa_fwd_ex(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                          int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                          float threshold_scale_factor, void* out, int32_t* skip_counter, uint32_t* decision_bitmap,
+                          float* tile_stat, void* stream) {
+  const Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
+               static_cast<cudaStream_t>(stream)};
+  return fwd_impl(a, threshold_scale_factor, skip_counter, decision_bitmap, tile_stat);
+}
+
+extern "C" int ssa_calibrate(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                             int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                             const float* thresholds, int n_thresholds, void* out, int32_t* counts, void* stream) {
+  const Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
+               static_cast<cudaStream_t>(stream)};
+  int rc = validate(a);
+  if (rc != SSA_OK) return rc;
+  if (!thresholds || !counts || n_thresholds < 1 || n_thresholds > SSA_MAX_THRESHOLDS) return SSA_ERR_INVALID_ARG;
+  for (int i = 0; i < n_thresholds; ++i)
+    if (!(thresholds[i] > 0.f) || std::isinf(thresholds[i])) return SSA_ERR_INVALID_ARG;
+  if (total_tokens == 0) return SSA_OK;
+  Params p = base_params(a);
+  p.counts = counts;
+  p.n_cal = n_thresholds;
+  for (int i = 0; i < n_thresholds; ++i) p.Lcal[i] = static_cast<float>(std::log2(static_cast<double>(thresholds[i])));
+  return dispatch_d<kCalib, false>(a, p);
+}
+
+extern "C" int ssa_get_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SSA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return SSA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return SSA_ERR_CUDA;
+  }
+  if (v & kStatusTimeout) return SSA_ERR_TIMEOUT;
+  if (v & kStatusDeviceArg) return SSA_ERR_DEVICE_ARG;
+  return SSA_OK;
+}

@@ -1,0 +1,147 @@
+/*
+ * ssa.h -- C ABI of the BLASST skip-softmax attention library for NVIDIA
+ * B200 (sm_100a).
+ *
+ * The method (Model-Optimizer README "Skip-Softmax Sparse Attention for
+ * Diffusion Models", introduction and "Threshold Modes"; Model-Optimizer
+ * commit page, "Triton kernels"): non-causal FlashAttention over 128 x 128
+ * tiles in which a KV tile whose scores all sit far below the running softmax
+ * max is skipped outright -- no V load, no exponentials, no accumulation.
+ * "Far below" is log2(lambda) in the log2 score domain, with
+ * lambda = threshold_scale_factor / seq_len_kv computed per sequence
+ * (README, "Threshold Modes", calibrated row; TRT-LLM VisualGen docs,
+ * "Skip Softmax Attention": the kernel consumes threshold_scale_factor and
+ * combines it with the sequence length at run time).
+ *
+ * Rules this library fixes where the pages are silent:
+ *   s2[r,c]  = fp32(q_r . k_c) * fp32(softmax_scale * log2 e)
+ *   d_j      = max over valid rows r of fp32(max_c s2[r,c] - m_r), where m_r
+ *              is the running max over the KV tiles kept BEFORE tile j
+ *              (d_0 = +inf); columns past the sequence end count as -inf and
+ *              rows past it do not vote;
+ *   skip j  <=> d_j < L, L = fp32(log2(threshold_scale_factor / S_kv));
+ *   threshold_scale_factor <= 0 disables skipping (L = -inf).
+ *
+ * Layout. Q, K, V and out are bf16, packed varlen [total_tokens, H, D]
+ * (row-major, D contiguous), D in {64, 128}; sequence b occupies rows
+ * cu_seqlens[b] .. cu_seqlens[b+1]-1 (self-attention: S_q = S_kv). Its query
+ * blocks are 128 rows each; the "global q-block" index numbers them over the
+ * batch in order (sequence 0's blocks first). Per-unit outputs are indexed
+ * [head][global q-block]; ssa_num_qblocks() gives their count Q.
+ *
+ * Ownership and streams. Every pointer argument is caller-owned; device
+ * pointers must stay valid until the work on `stream` completes. `stream` is
+ * a cudaStream_t (NULL = legacy default stream). The compute entry points
+ * validate their arguments on the host, return a negative status before any
+ * launch when they are wrong, enqueue work on `stream` and return without
+ * synchronising. Errors a kernel detects (an inconsistent cu_seqlens, a
+ * device wait that ran past its time limit) are recorded in a per-device
+ * status word that ssa_get_error() reads. Q, K, V and out must be 16-byte
+ * aligned.
+ */
+#ifndef SSA_H_
+#define SSA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  SSA_OK = 0,
+  SSA_ERR_INVALID_ARG = -1, /* bad pointer, size or value (host check)      */
+  SSA_ERR_UNSUPPORTED = -2, /* head_dim not 64/128, misaligned pointer      */
+  SSA_ERR_CUDA = -3,        /* a CUDA runtime or launch error               */
+  SSA_ERR_TIMEOUT = -4,     /* a device-side wait exceeded its time limit   */
+  SSA_ERR_DEVICE_ARG = -5   /* the kernel found cu_seqlens inconsistent     */
+};
+
+#define SSA_TILE 128          /* Br = Bc = 128                                 */
+#define SSA_MAX_THRESHOLDS 32 /* most thresholds one calibration call counts  */
+
+/*
+ * Skip-softmax attention forward (commit page, "Triton kernels": the
+ * inference kernel with tile skipping and runtime sparsity counters).
+ *   q, k, v      device bf16 [total_tokens, num_heads, head_dim]
+ *   cu_seqlens   device int32 [batch + 1], non-decreasing, cu_seqlens[batch]
+ *                <= total_tokens
+ *   max_seqlen   >= every sequence length (sizes the debug outputs)
+ *   softmax_scale   <= 0 selects 1/sqrt(head_dim)
+ *   threshold_scale_factor  lambda * S_kv; <= 0 runs dense attention
+ *   out          device bf16 [total_tokens, num_heads, head_dim]; rows of
+ *                every sequence are written, nothing else is touched
+ *   skip_counter device int32 [num_heads][Q] or NULL: tiles skipped per unit
+ *                (plain stores, no atomics)
+ * Returns SSA_OK or a negative status.
+ */
+int ssa_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch, int total_tokens,
+            int max_seqlen, int num_heads, int head_dim, float softmax_scale, float threshold_scale_factor,
+            void* out, int32_t* skip_counter, void* stream);
+
+/*
+ * ssa_fwd plus per-tile diagnostics, for tests. T = ceil(max_seqlen / 128).
+ *   decision_bitmap  device uint32 [num_heads][Q][ceil(T/32)] or NULL: bit
+ *                    (j & 31) of word (j >> 5) is 1 when KV tile j was skipped
+ *   tile_stat        device float [num_heads][Q][T] or NULL: the statistic
+ *                    d_j of every tile (+inf for tile 0; entries past the
+ *                    sequence's last tile are left untouched)
+ * With threshold_scale_factor <= 0 the statistics follow the dense trajectory.
+ */
+int ssa_fwd_ex(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch, int total_tokens,
+               int max_seqlen, int num_heads, int head_dim, float softmax_scale, float threshold_scale_factor,
+               void* out, int32_t* skip_counter, uint32_t* decision_bitmap, float* tile_stat, void* stream);
+
+/*
+ * Calibration pass (commit page, "Triton kernels": full attention that counts
+ * how many tiles would be skipped at each of N thresholds at once, with
+ * per-program output buffers and no atomics; threshold trials from
+ * Model-Optimizer PR #1166, "Usage").
+ *   thresholds    HOST float [n_thresholds], raw lambda values (> 0), each
+ *                 compared as log2(lambda); 1 <= n_thresholds <= 32
+ *   out           device bf16, the dense attention output
+ *   counts        device int32 [num_heads][Q][n_thresholds]: per unit, the
+ *                 number of KV tiles j >= 1 with d_j < log2(lambda_k) on the
+ *                 dense trajectory. For lambda_k <= 1 this equals ssa_fwd's
+ *                 skip count at threshold_scale_factor = lambda_k * S_kv.
+ */
+int ssa_calibrate(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                  int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                  const float* thresholds, int n_thresholds, void* out, int32_t* counts, void* stream);
+
+/*
+ * threshold_scale_factor = a * exp(b * target_sparsity) (README, "Calibrated
+ * threshold"; TRT-LLM VisualGen docs, "Checkpoint Config"). Returns NaN when
+ * a <= 0, target_sparsity is outside [0, 1] or an argument is not finite.
+ * A caller holding log_a passes exp(log_a).
+ */
+double ssa_resolve(double a, double b, double target_sparsity);
+
+/*
+ * Log-space least-squares fit of ln(scale_factor) = ln(a) + b * sparsity
+ * (commit page, "Calibration": fit_logspace minimises relative error and the
+ * observed sparsity range is recorded for extrapolation warnings). Points
+ * with sparsity outside (0, 1) or scale_factor <= 0 are ignored. Writes a, b
+ * and the observed [s_min, s_max] of the points used. Host arrays. Returns
+ * SSA_OK, or SSA_ERR_INVALID_ARG when fewer than two distinct usable
+ * sparsities remain or a pointer is NULL.
+ */
+int ssa_fit_logspace(const double* sparsity, const double* scale_factor, int n, double* a, double* b, double* s_min,
+                     double* s_max);
+
+/* Number of 128-row query blocks Q over the batch, from a HOST copy of
+ * cu_seqlens; negative status when it is inconsistent. */
+int ssa_num_qblocks(const int32_t* cu_seqlens_host, int batch);
+
+/* Synchronise `stream`, then return and clear this device's kernel status:
+ * SSA_OK, SSA_ERR_TIMEOUT, SSA_ERR_DEVICE_ARG or SSA_ERR_CUDA. */
+int ssa_get_error(void* stream);
+
+/* Static description of a status code. */
+const char* ssa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSA_H_ */

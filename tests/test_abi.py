@@ -1,0 +1,109 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+entry point include/ssa.h declares, rejects bad arguments on the host before
+touching CUDA, and its host-side math agrees with the oracle."""
+import ctypes
+import math
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from tests.golden import first
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_entry_points():
+    text = open(os.path.join(ROOT, "include", "ssa.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:int|double|const char\*)\s+(ssa_\w+)\s*\(", text, re.M)))
+
+
+@pytest.fixture(scope="module")
+def ssa():
+    from block_sparse_flashattention_ssa_b200 import build
+
+    build.build()
+    import block_sparse_flashattention_ssa_b200 as m
+
+    return m
+
+
+def test_library_exports_every_declared_symbol(ssa):
+    names = declared_entry_points()
+    assert {"ssa_fwd", "ssa_fwd_ex", "ssa_calibrate", "ssa_resolve", "ssa_fit_logspace"} <= set(names)
+    out = subprocess.check_output(["nm", "-D", "--defined-only", ssa.library_path()], text=True)
+    exported = set(re.findall(r" T (ssa_\w+)$", out, re.M))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(ssa.lib(), n)
+
+
+def test_library_is_built_for_sm100a(ssa):
+    out = subprocess.run(["cuobjdump", "--list-elf", ssa.library_path()], capture_output=True, text=True).stdout
+    assert "sm_100a" in out
+
+
+def test_host_argument_validation(ssa):
+    L = ssa.lib()
+    fake = ctypes.c_void_p(0x10000)
+    mis = ctypes.c_void_p(0x10008)
+    none = None
+    args = dict(q=fake, k=fake, v=fake, cu=fake, batch=1, total=256, maxs=256, H=2, D=128, scale=0.0, tsf=0.0,
+                out=fake, sc=None, stream=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return L.ssa_fwd(a["q"], a["k"], a["v"], a["cu"], a["batch"], a["total"], a["maxs"], a["H"], a["D"],
+                         a["scale"], a["tsf"], a["out"], a["sc"], a["stream"])
+
+    assert call(q=none) == ssa.SSA_ERR_INVALID_ARG
+    assert call(out=none) == ssa.SSA_ERR_INVALID_ARG
+    assert call(batch=0) == ssa.SSA_ERR_INVALID_ARG
+    assert call(total=-1) == ssa.SSA_ERR_INVALID_ARG
+    assert call(H=0) == ssa.SSA_ERR_INVALID_ARG
+    assert call(D=96) == ssa.SSA_ERR_UNSUPPORTED
+    assert call(D=256) == ssa.SSA_ERR_UNSUPPORTED
+    assert call(k=mis) == ssa.SSA_ERR_UNSUPPORTED
+    assert call(tsf=float("nan")) == ssa.SSA_ERR_INVALID_ARG
+    assert call(tsf=float("inf")) == ssa.SSA_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == ssa.SSA_ERR_INVALID_ARG
+    assert call(total=0) == ssa.SSA_OK  # nothing to do, nothing launched
+    th = np.array([1e-3, 0.5], dtype=np.float32)
+    cal = lambda th, n, counts=fake: L.ssa_calibrate(fake, fake, fake, fake, 1, 256, 256, 2, 128, 0.0,
+                                                     th.ctypes.data if th is not None else None, n, fake, counts,
+                                                     None)
+    assert cal(th, 0) == ssa.SSA_ERR_INVALID_ARG
+    assert cal(th, 33) == ssa.SSA_ERR_INVALID_ARG
+    assert cal(None, 2) == ssa.SSA_ERR_INVALID_ARG
+    assert cal(th, 2, counts=None) == ssa.SSA_ERR_INVALID_ARG
+    assert cal(np.array([1e-3, 0.0], dtype=np.float32), 2) == ssa.SSA_ERR_INVALID_ARG
+    ex = L.ssa_fwd_ex(fake, fake, fake, fake, 1, 256, 0, 2, 128, 0.0, 10.0, fake, None, fake, None, None)
+    assert ex == ssa.SSA_ERR_INVALID_ARG  # diagnostics need max_seqlen >= 1
+    assert ssa.lib().ssa_status_string(ssa.SSA_ERR_TIMEOUT)
+
+
+def test_num_qblocks(ssa):
+    assert ssa.num_qblocks([0, 1, 129, 129, 385]) == 1 + 1 + 0 + 2  # lengths 1, 128, 0, 256
+    assert ssa.num_qblocks([0, 75600]) == 591
+    with pytest.raises(ssa.SSAError):
+        ssa.num_qblocks([0, 10, 5])
+
+
+def test_resolve_and_fit_match_oracle(ssa):
+    for a, b in first("page_constants.txt", "formula"):
+        for s in [0.0, 0.25, 0.5, 0.7, 0.9, 1.0]:
+            assert ssa.resolve(a, b, s) == oracle.resolve(a, b, s)
+    assert math.isnan(ssa.resolve(0.0, 1.0, 0.5)) and math.isnan(ssa.resolve(1.0, 1.0, -0.1))
+    rng = np.random.default_rng(1)
+    s = rng.uniform(0.0, 1.0, 50)
+    s[:3] = [0.0, 1.0, 0.0]
+    sf = 3e-4 * np.exp(7.5 * s) * np.exp(rng.normal(0, 0.2, 50))
+    got = ssa.fit_logspace(s, sf)
+    ref = oracle.fit_logspace(s, sf)
+    np.testing.assert_allclose(got, ref, rtol=1e-12)
+    with pytest.raises(ssa.SSAError):
+        ssa.fit_logspace([0.5, 0.5], [1.0, 1.0])
