@@ -39,7 +39,10 @@ SSA_ERR_DEVICE_ARG = -5
 class SSAError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {status} ({_lib.ssa_status_string(status).decode()})")
+        detail = ""
+        if status == SSA_ERR_CUDA:
+            detail = f": {_lib.ssa_last_cuda_error().decode()}"
+        super().__init__(f"{what}: {status} ({_lib.ssa_status_string(status).decode()}{detail})")
 
 
 def _load():
@@ -63,6 +66,8 @@ def _load():
     L.ssa_get_error.argtypes = [vp]
     L.ssa_status_string.restype = ctypes.c_char_p
     L.ssa_status_string.argtypes = [i32]
+    L.ssa_last_cuda_error.restype = ctypes.c_char_p
+    L.ssa_last_cuda_error.argtypes = []
     return L
 
 

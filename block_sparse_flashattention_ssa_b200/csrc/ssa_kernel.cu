@@ -57,6 +57,12 @@ constexpr uint32_t kFull = 0xFFFFFFFFu;
 enum Mode : int { kDense = 0, kSkip = 1, kCalib = 2 };
 
 __device__ int g_status;  // sticky error bits of this device, read by ssa_get_error
+thread_local const char* t_last_cuda_error = "no error";
+
+int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = cudaGetErrorString(e);
+  return SSA_ERR_CUDA;
+}
 
 struct Params {
   const int32_t* cu_seqlens;
@@ -75,13 +81,14 @@ struct Params {
 struct Ctl {
   uint64_t bar_q;
   uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[2], s_free[2], p_ready[2], pv_done[2];
+  uint64_t v_full[kVStages];
+  uint64_t s_full[2], p_ready[2], pv_done[2];  // pv_done[b] also frees V stage b
   uint64_t dec_ready[kDecRing], red_bar[2], drain;
   uint32_t tmem_base;
   int abort_flag;
   int dec[kDecRing];
   float red[2][4];
+  int cnt[SSA_MAX_THRESHOLDS];  // calibration counts of this unit (thread 0 only)
   int seq, qb, S, start, gqb, nq_total;
 };
 
@@ -188,9 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto k_full = [&](int i) { return smem_u32(&ctl.k_full[i]); };
   auto k_empty = [&](int i) { return smem_u32(&ctl.k_empty[i]); };
   auto v_full = [&](int i) { return smem_u32(&ctl.v_full[i]); };
-  auto v_empty = [&](int i) { return smem_u32(&ctl.v_empty[i]); };
   auto s_full = [&](int i) { return smem_u32(&ctl.s_full[i]); };
-  auto s_free = [&](int i) { return smem_u32(&ctl.s_free[i]); };
   auto p_ready = [&](int i) { return smem_u32(&ctl.p_ready[i]); };
   auto pv_done = [&](int i) { return smem_u32(&ctl.pv_done[i]); };
   auto dec_ready = [&](int i) { return smem_u32(&ctl.dec_ready[i]); };
@@ -204,11 +209,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kVStages; ++i) {
       mbar_init(v_full(i), 1);
-      mbar_init(v_empty(i), 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
-      mbar_init(s_free(i), 128);
       mbar_init(p_ready(i), 128);
       mbar_init(pv_done(i), 1);
       mbar_init(red_bar(i), 4);
@@ -261,7 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!skip) {
           const int vs = v_issued % kVStages;
-          if (v_issued >= kVStages && !wait_bar(v_empty(vs), ((v_issued / kVStages) - 1) & 1, abort_flag)) {
+          // V stage vs was last read by PV number v_issued - 2, which commits to pv_done[vs]
+          if (v_issued >= kVStages && !wait_bar(pv_done(vs), ((v_issued / kVStages) - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -290,7 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = t % kKStages;
         if (!wait_bar(k_full(st), (t / kKStages) & 1, abort_flag)) return false;
         const int sb = t & 1;
-        if (t >= 2 && !wait_bar(s_free(sb), ((t >> 1) - 1) & 1, abort_flag)) return false;
+        // S buffer sb last held S_{t-2}; the softmax finished reading it before
+        // arriving on p_ready for tile t-2, which this thread has already waited for.
         tc_fence_after();
         const uint32_t k_s = smem_u32(smem + L::kK + st * L::kTileBytes);
         const uint32_t d_tmem = tmem + (sb ? kColS1 : kColS0);
@@ -330,7 +335,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + kColO, p_tmem + ks * 8, smem_desc_sw128(v_s + ks * 16 * 128, L::kChunkBytes, 1024),
                  idesc_pv, (kept > 0 || ks > 0) ? 1u : 0u);
         }
-        tc_commit(v_empty(vs));
         tc_commit(pv_done(kept & 1));
         ++kept;
       }
@@ -351,9 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_used = -INFINITY;  // reference max of the exponentials (lags m_true by < kRescaleThreshold)
     float l = 0.f;
     int kept = 0, nskip = 0;
-    int cnt[SSA_MAX_THRESHOLDS];
-#pragma unroll
-    for (int k = 0; k < SSA_MAX_THRESHOLDS; ++k) cnt[k] = 0;
+    if (MODE == kCalib && threadIdx.x == 0)
+      for (int k = 0; k < SSA_MAX_THRESHOLDS; ++k) ctl.cnt[k] = 0;
     uint32_t bits = 0;
     bool ok = true;
 
@@ -363,8 +366,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld_x128(lane_base + (sb ? kColS1 : kColS0), sr);
-      tc_fence_before();
-      mbar_arrive(s_free(sb));
       float s[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
@@ -396,9 +397,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         volatile float* red = ctl.red[sb];
         const float d = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
         if (MODE == kSkip) skip = d < Lthr;
-        if (MODE == kCalib) {
-#pragma unroll
-          for (int k = 0; k < SSA_MAX_THRESHOLDS; ++k) cnt[k] += (k < p.n_cal && d < p.Lcal[k]) ? 1 : 0;
+        if (MODE == kCalib && threadIdx.x == 0) {
+          for (int k = 0; k < p.n_cal; ++k) ctl.cnt[k] += d < p.Lcal[k] ? 1 : 0;
         }
         if (EX && threadIdx.x == 0) {
           if (p.tile_stat) p.tile_stat[unit * p.max_tiles + j] = d;
@@ -451,7 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         pk[i] = pack_bf16x2(p0, p1);
       }
       l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      if (kept >= 2 && !(ok = warp_wait(pv_done(kept & 1), ((kept - 2) >> 1) & 1, abort_flag))) break;
+      // P buffer kept & 1 was last read by the PV two kept tiles back, which
+      // was issued before S_j and so completed before S_j did.
       tmem_st_x64(lane_base + ((kept & 1) ? kColP1 : kColP0), pk);
       tc_fence_before();
       mbar_arrive(p_ready(sb));
@@ -482,9 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (threadIdx.x == 0) {
         if (p.skip_counter) p.skip_counter[unit] = nskip;
         if (MODE == kCalib) {
-#pragma unroll
-          for (int k = 0; k < SSA_MAX_THRESHOLDS; ++k)
-            if (k < p.n_cal) p.counts[unit * p.n_cal + k] = cnt[k];
+          for (int k = 0; k < p.n_cal; ++k) p.counts[unit * p.n_cal + k] = ctl.cnt[k];
         }
       }
     }
@@ -569,15 +568,19 @@ template <int D, int MODE, bool EX>
 int launch(const Call& a, const Params& p) {
   CUtensorMap tq, tk, tv;
   if (!make_tensor_map(&tq, a.q, a.total_tokens, a.H, D) || !make_tensor_map(&tk, a.k, a.total_tokens, a.H, D) ||
-      !make_tensor_map(&tv, a.v, a.total_tokens, a.H, D))
+      !make_tensor_map(&tv, a.v, a.total_tokens, a.H, D)) {
+    t_last_cuda_error = "cuTensorMapEncodeTiled failed or the driver entry point is unavailable";
     return SSA_ERR_CUDA;
+  }
   auto kernel = ssa_attention_kernel<D, MODE, EX>;
   constexpr int smem = Layout<D>::kAlloc;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return SSA_ERR_CUDA;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return cuda_fail(e);
+  // one CTA per query block: sum over sequences of ceil(S_b / 128) <= ceil(T / 128) + batch
   const dim3 grid(static_cast<unsigned>((a.total_tokens + kBM - 1) / kBM + a.batch), static_cast<unsigned>(a.H));
   kernel<<<grid, kThreads, smem, a.stream>>>(tq, tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? SSA_OK : SSA_ERR_CUDA;
+  e = cudaGetLastError();
+  return e == cudaSuccess ? SSA_OK : cuda_fail(e);
 }
 
 template <int MODE, bool EX>
@@ -641,13 +644,18 @@ extern "C" int ssa_calibrate(const void* q, const void* k, const void* v, const 
   return dispatch_d<kCalib, false>(a, p);
 }
 
+extern "C" const char* ssa_last_cuda_error(void) { return t_last_cuda_error; }
+
 extern "C" int ssa_get_error(void* stream) {
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SSA_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
   int v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return SSA_ERR_CUDA;
+  e = cudaMemcpyFromSymbol(&v, g_status, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
   if (v != 0) {
     const int zero = 0;
-    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return SSA_ERR_CUDA;
+    e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
   }
   if (v & kStatusTimeout) return SSA_ERR_TIMEOUT;
   if (v & kStatusDeviceArg) return SSA_ERR_DEVICE_ARG;

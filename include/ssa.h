@@ -140,6 +140,10 @@ int ssa_get_error(void* stream);
 /* Static description of a status code. */
 const char* ssa_status_string(int status);
 
+/* Text of the last CUDA error this library saw on the calling host thread
+ * (the cause behind an SSA_ERR_CUDA); "no error" if none. Static storage. */
+const char* ssa_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif
