@@ -48,6 +48,33 @@ def peaks():
         return 1590.0, 1400.0, 6650.0, "fallback"
 
 
+def kernel_source_hash() -> str:
+    """sha256 (first 16 hex) of the kernel sources, to match committed ncu counters."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in ("ssa_kernel.cu", "sm100.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_flashattention_ssa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str, tsf: float):
+    """DRAM bytes per launch (read + write) from a committed ncu capture of
+    this exact kernel source, workload and threshold; None otherwise."""
+    path = os.path.join(ROOT, "profiles", "ssa_attention_wan14b_dram.md")
+    if not os.path.exists(path):
+        return None
+    want = kernel_source_hash()
+    for line in open(path):
+        if not line.startswith("traffic:"):
+            continue
+        kv = dict(x.split("=", 1) for x in line.split()[1:])
+        if kv.get("hash") == want and kv.get("workload") == workload and abs(float(kv["tsf"]) - tsf) <= 1e-6 * max(1.0, tsf):
+            return float(kv["bytes"])
+    return None
+
+
 def tiles_of(seqlens, H):
     return sum(((s + TILE - 1) // TILE) ** 2 for s in seqlens) * H
 
@@ -295,7 +322,7 @@ def run_ours(args):
         "fit": fit,
         "targets": rows,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": p_burst, "unit": "TFLOP/s",
-                     "frac": achieved / p_burst, "traffic": None,
+                     "frac": achieved / p_burst, "traffic": measured_traffic(args.workload, tsf),
                      "peak_kind": f"{peak_kind} bf16 burst", "peak_sustained": p_sus,
                      "frac_sustained": achieved / p_sus,
                      "dense_frac": rows["dense"]["dense_eq_tflops"] / p_burst if dense_ms else achieved / p_burst},
@@ -373,6 +400,61 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_calib_sweep(args):
+    """Calibration over seeds x positional amplitudes on the S = 75,600 shape:
+    ssa_calibrate at the 16 raw-lambda trials on each input, one log-space
+    fit over all points, then the forward at the resolved targets on the
+    first input (achieved vs target sparsity)."""
+    import torch
+
+    import block_sparse_flashattention_ssa_b200 as ssa
+    import synth
+
+    dev = torch.device("cuda", 0)
+    base = getattr(synth, WORKLOADS[args.workload])
+    lams = synth.CALIB_THRESHOLDS
+    S = base.seqlens[0]
+    tiles = tiles_of(base.seqlens, base.H)
+    pts_s, pts_sf, runs, first = [], [], [], None
+    for seed in synth.CALIB_SEEDS:
+        for amp in synth.CALIB_AMPS:
+            w = synth.Workload(base.name, base.grids, H=base.H, D=base.D, seed=seed, amp=amp)
+            q, k, v = synth.generate(w)
+            to_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+            dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+            dcu = torch.from_numpy(w.cu_seqlens).to(dev)
+            ssa.calibrate(dq, dk, dv, dcu, w.max_seqlen, lams)  # warm
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            _, counts = ssa.calibrate(dq, dk, dv, dcu, w.max_seqlen, lams)
+            e1.record()
+            ssa.check_device()
+            sp = counts.sum(dim=(0, 1)).double().cpu().numpy() / tiles
+            runs.append({"seed": seed, "amp": amp, "calib_ms": e0.elapsed_time(e1),
+                         "sparsity": [round(float(x), 5) for x in sp]})
+            pts_s += list(sp)
+            pts_sf += [lam * S for lam in lams]
+            if first is None and seed == base.seed and amp == base.amp:
+                first = (dq, dk, dv, dcu, w)  # the benchmark input: targets are checked on it
+            else:
+                del dq, dk, dv
+    a, b, smin, smax = ssa.fit_logspace(pts_s, pts_sf)
+    dq, dk, dv, dcu, w = first
+    skip = torch.zeros((w.H, ssa.num_qblocks(w.cu_seqlens)), dtype=torch.int32, device=dev)
+    achieved = {}
+    for s_t in TARGETS:
+        tsf = ssa.resolve(a, b, s_t)
+        ssa.fwd(dq, dk, dv, dcu, w.max_seqlen, tsf, skip_counter=skip)
+        ssa.check_device()
+        achieved[str(s_t)] = {"tsf": tsf, "achieved_sparsity": float(skip.sum().item()) / tiles}
+    print(json.dumps({"metric": "calibration sweep: fit of threshold_scale_factor = a*exp(b*s)",
+                      "config": {"workload": base.name, "seeds": synth.CALIB_SEEDS, "amps": synth.CALIB_AMPS,
+                                 "thresholds": lams},
+                      "fit": {"a": a, "b": b, "s_min": smin, "s_max": smax, "points": len(pts_s)},
+                      "calib_ms_mean": statistics.mean(r["calib_ms"] for r in runs),
+                      "targets_on_benchmark_input": achieved, "runs": runs}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -383,11 +465,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="wan14b", choices=sorted(WORKLOADS),
                     help="problem shape (the default is the benchmark workload; the others serve profiling)")
+    ap.add_argument("--calib-sweep", action="store_true",
+                    help="calibration over 4 seeds x 4 amplitudes, fit, and achieved vs target sparsity")
     ap.add_argument("--tsf", type=float, default=None,
                     help="fixed threshold_scale_factor: skip calibration and the side rows")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.calib_sweep:
+        run_calib_sweep(args)
     else:
         run_ours(args)
 

@@ -6,9 +6,9 @@
 //   warp 4  TMA producer: Q once, K tiles through a 3-stage ring, and V tiles
 //           through a 2-stage ring -- V of tile j only once the softmax warps
 //           have decided to keep tile j (skipped tiles issue no V load);
-//   warp 5  tcgen05 issuer: S_j = Q K_j^T into one of two TMEM S buffers
-//           (issued one tile ahead), and O += P_j V_j from a TMEM copy of P_j
-//           (kept tiles only);
+//   warp 5  tcgen05 issuer: once P_j is ready, O += P_j V_j (kept tiles only,
+//           P_j read from TMEM) and then S_{j+2} = Q K_{j+2}^T into the S
+//           buffer S_j has just freed (two TMEM S buffers, S two tiles ahead);
 //   warps 0-3  softmax, one query row per thread: row max of S_j in the log2
 //           domain, the CTA-wide skip vote d_j < log2(lambda) (Model-Optimizer
 //           commit page, "Triton kernels": tiles whose max score is far below
@@ -53,6 +53,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kStatusTimeout = 1;
 constexpr int kStatusDeviceArg = 2;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
+constexpr int kVoteBarrier = 1;  // named barrier of the four softmax warps (0 is __syncthreads)
 
 enum Mode : int { kDense = 0, kSkip = 1, kCalib = 2 };
 
@@ -83,7 +84,7 @@ struct Ctl {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages];
   uint64_t s_full[2], p_ready[2], pv_done[2];  // pv_done[b] also frees V stage b
-  uint64_t dec_ready[kDecRing], red_bar[2], drain;
+  uint64_t dec_ready[kDecRing], s_free[2], drain;
   uint32_t tmem_base;
   int abort_flag;
   int dec[kDecRing];
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto p_ready = [&](int i) { return smem_u32(&ctl.p_ready[i]); };
   auto pv_done = [&](int i) { return smem_u32(&ctl.pv_done[i]); };
   auto dec_ready = [&](int i) { return smem_u32(&ctl.dec_ready[i]); };
-  auto red_bar = [&](int i) { return smem_u32(&ctl.red_bar[i]); };
+  auto s_free = [&](int i) { return smem_u32(&ctl.s_free[i]); };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(s_full(i), 1);
       mbar_init(p_ready(i), 128);
       mbar_init(pv_done(i), 1);
-      mbar_init(red_bar(i), 4);
+      mbar_init(s_free(i), 128);
     }
     for (int i = 0; i < kDecRing; ++i) mbar_init(dec_ready(i), 1);
     mbar_init(smem_u32(&ctl.drain), 1);
@@ -290,13 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
       const uint32_t q_s = smem_u32(smem + L::kQ);
-      auto issue_qk = [&](int t) -> bool {
+      // S_t = Q K_t^T into S buffer t & 1 (no waits inside: the caller has made
+      // sure K_t has landed and the buffer's previous S was consumed).
+      auto issue_qk = [&](int t) {
         const int st = t % kKStages;
-        if (!wait_bar(k_full(st), (t / kKStages) & 1, abort_flag)) return false;
         const int sb = t & 1;
-        // S buffer sb last held S_{t-2}; the softmax finished reading it before
-        // arriving on p_ready for tile t-2, which this thread has already waited for.
-        tc_fence_after();
         const uint32_t k_s = smem_u32(smem + L::kK + st * L::kTileBytes);
         const uint32_t d_tmem = tmem + (sb ? kColS1 : kColS0);
 #pragma unroll
@@ -309,34 +308,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(s_full(sb));
         tc_commit(k_empty(st));
-        return true;
       };
       bool ok = wait_bar(bar_q, 0, abort_flag);
-      if (ok) {
+      for (int t = 0; ok && t < 2 && t < nkv; ++t) {  // S_0 and S_1
+        if (!(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag))) break;
         tc_fence_after();
-        ok = issue_qk(0);
+        issue_qk(t);
       }
-      int kept = 0;
-      for (int j = 0; ok && j < nkv; ++j) {
-        if (j + 1 < nkv && !(ok = issue_qk(j + 1))) break;
-        if (!(ok = wait_bar(p_ready(j & 1), (j >> 1) & 1, abort_flag))) break;
-        tc_fence_after();
-        const bool skip = (MODE == kSkip) && reinterpret_cast<volatile int*>(ctl.dec)[j % kDecRing] != 0;
-        if (skip) continue;
-        const int vs = kept % kVStages;
-        if (!(ok = wait_bar(v_full(vs), (kept / kVStages) & 1, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t p_tmem = tmem + ((kept & 1) ? kColP1 : kColP0);
+      // O += P_j V_j from the TMEM copy of P_j and V stage vs.
+      auto issue_pv = [&](int kp, int vs) {
+        const uint32_t p_tmem = tmem + ((kp & 1) ? kColP1 : kColP0);
         const uint32_t v_s = smem_u32(smem + L::kV + vs * L::kTileBytes);
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks) {
           // V is MN-major (d contiguous): 16 kv rows = 2 KB per k step; the
           // second 64-column chunk of d sits one 16 KB chunk further (LBO).
           mma_ts(tmem + kColO, p_tmem + ks * 8, smem_desc_sw128(v_s + ks * 16 * 128, L::kChunkBytes, 1024),
-                 idesc_pv, (kept > 0 || ks > 0) ? 1u : 0u);
+                 idesc_pv, (kp > 0 || ks > 0) ? 1u : 0u);
         }
-        tc_commit(pv_done(kept & 1));
-        ++kept;
+        tc_commit(pv_done(kp & 1));
+      };
+      int kept = 0;
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int t = j + 2;  // S_{j+2} goes to S_j's buffer
+        if (MODE == kSkip) {
+          // Skipped tiles are short, so S_{j+2} is issued as soon as the
+          // softmax has loaded S_j, before waiting for P_j.
+          if (t < nkv) {
+            if (!(ok = wait_bar(s_free(j & 1), (j >> 1) & 1, abort_flag))) break;
+            if (!(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_qk(t);
+          }
+          if (!(ok = wait_bar(p_ready(j & 1), (j >> 1) & 1, abort_flag))) break;
+          if (reinterpret_cast<volatile int*>(ctl.dec)[j % kDecRing] != 0) continue;
+          const int vs = kept % kVStages;
+          if (!(ok = wait_bar(v_full(vs), (kept / kVStages) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(kept, vs);
+          ++kept;
+        } else {
+          // Wait once for everything O += P_j V_j and S_{j+2} need, then issue
+          // both groups back to back: tcgen05.mma issue is nearly synchronous,
+          // so each wait on this thread is a tensor-pipe bubble. The softmax
+          // finished reading S_j before arriving on p_ready for tile j.
+          if (!(ok = wait_bar(p_ready(j & 1), (j >> 1) & 1, abort_flag))) break;
+          const int vs = kept % kVStages;
+          if (!(ok = wait_bar(v_full(vs), (kept / kVStages) & 1, abort_flag))) break;
+          if (t < nkv && !(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(kept, vs);
+          ++kept;
+          if (t < nkv) issue_qk(t);
+        }
       }
       if (!ok) {  // let every MMA issued so far finish before TMEM is released
         tc_commit(smem_u32(&ctl.drain));
@@ -366,6 +390,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld_x128(lane_base + (sb ? kColS1 : kColS0), sr);
+      if (MODE == kSkip) {
+        tc_fence_before();
+        mbar_arrive(s_free(sb));
+      }
       float s[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
@@ -389,11 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float dr = row_valid ? (tmax - m_true) : -INFINITY;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) dr = fmaxf(dr, __shfl_xor_sync(kFull, dr, o));
-        if (lane == 0) {
-          ctl.red[sb][warp] = dr;
-          mbar_arrive(red_bar(sb));
-        }
-        if (!(ok = warp_wait(red_bar(sb), (j >> 1) & 1, abort_flag))) break;
+        if (lane == 0) ctl.red[sb][warp] = dr;
+        named_barrier_sync(kVoteBarrier, 128);
         volatile float* red = ctl.red[sb];
         const float d = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
         if (MODE == kSkip) skip = d < Lthr;
@@ -451,13 +476,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         pk[i] = pack_bf16x2(p0, p1);
       }
       l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      // P buffer kept & 1 was last read by the PV two kept tiles back, which
-      // was issued before S_j and so completed before S_j did.
+      // P buffer kept & 1 was last read by the PV two kept tiles back. In the
+      // dense and calibration order that PV was issued before S_j and so
+      // completed before S_j did; in skip mode S is issued ahead of PV, so wait.
+      if (MODE == kSkip && kept >= 2 &&
+          !(ok = warp_wait(pv_done(kept & 1), ((kept - 2) >> 1) & 1, abort_flag)))
+        break;
       tmem_st_x64(lane_base + ((kept & 1) ? kColP1 : kColP0), pk);
       tc_fence_before();
       mbar_arrive(p_ready(sb));
       ++kept;
     }
+
+    // A warp that left the loop on an error arrives once on the vote barrier,
+    // so the other softmax warps cannot be left waiting at it: the barrier is
+    // a full barrier per tile, so no warp is ever more than one instance away.
+    if (!ok && (MODE != kDense || EX)) named_barrier_arrive(kVoteBarrier, 128);
 
     // Epilogue: O / l -> bf16, masked row stores; per-unit counters.
     if (ok && kept > 0) ok = warp_wait(pv_done((kept - 1) & 1), ((kept - 1) >> 1) & 1, abort_flag);
