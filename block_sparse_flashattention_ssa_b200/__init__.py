@@ -68,6 +68,8 @@ def _load():
     L.ssa_status_string.argtypes = [i32]
     L.ssa_last_cuda_error.restype = ctypes.c_char_p
     L.ssa_last_cuda_error.argtypes = []
+    L.ssa_wait_timeout_check.restype = i32
+    L.ssa_wait_timeout_check.argtypes = [vp, ctypes.c_int64, vp]
     return L
 
 
@@ -176,6 +178,18 @@ def fit_logspace(sparsity, scale_factor):
     _check(_lib.ssa_fit_logspace(s.ctypes.data, sf.ctypes.data, len(s), *[ctypes.byref(o) for o in out]),
            "ssa_fit_logspace")
     return tuple(o.value for o in out)
+
+
+def wait_timeout_check(limit_ns: int = 20_000_000, stream=None):
+    """Diagnostic: run the kernels' bounded wait on a barrier nothing arrives
+    on. Returns (completed, abort_flag, microseconds_waited) from the device;
+    the device status then holds SSA_ERR_TIMEOUT (read it with get_error)."""
+    import torch
+
+    res = torch.full((3,), -1, dtype=torch.int32, device="cuda")
+    _check(_lib.ssa_wait_timeout_check(_ptr(res), int(limit_ns), _stream_handle(stream)), "ssa_wait_timeout_check")
+    torch.cuda.synchronize()
+    return tuple(int(x) for x in res.cpu().tolist())
 
 
 def get_error(stream=None) -> int:

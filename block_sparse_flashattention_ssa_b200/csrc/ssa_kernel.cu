@@ -105,20 +105,30 @@ struct Layout {
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B (128B swizzle atoms)
 };
 
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                         uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 31u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(&g_status, kStatusTimeout);
         return false;
       }
     }
   }
+}
+
+// One arrival for the whole warp: order this warp's finished tcgen05 loads
+// and stores before the thread synchronisation, gather the warp, and let
+// lane 0 arrive (one atomic on the barrier word instead of 32).
+__device__ __forceinline__ void warp_arrive(uint32_t bar, int lane) {
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
 }
 
 // Warp-uniform bounded wait: every lane returns the same verdict.
@@ -213,9 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
-      mbar_init(p_ready(i), 128);
+      mbar_init(p_ready(i), 4);  // one arrival per softmax warp
       mbar_init(pv_done(i), 1);
-      mbar_init(s_free(i), 128);
+      mbar_init(s_free(i), 4);
     }
     for (int i = 0; i < kDecRing; ++i) mbar_init(dec_ready(i), 1);
     mbar_init(smem_u32(&ctl.drain), 1);
@@ -390,10 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld_x128(lane_base + (sb ? kColS1 : kColS0), sr);
-      if (MODE == kSkip) {
-        tc_fence_before();
-        mbar_arrive(s_free(sb));
-      }
+      if (MODE == kSkip) warp_arrive(s_free(sb), lane);
       float s[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
@@ -414,9 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       bool skip = false;
       if (MODE != kDense || EX) {
-        float dr = row_valid ? (tmax - m_true) : -INFINITY;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) dr = fmaxf(dr, __shfl_xor_sync(kFull, dr, o));
+        const float dr = warp_max_f32(row_valid ? (tmax - m_true) : -INFINITY);
         if (lane == 0) ctl.red[sb][warp] = dr;
         named_barrier_sync(kVoteBarrier, 128);
         volatile float* red = ctl.red[sb];
@@ -440,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (skip) {
         ++nskip;
-        mbar_arrive(p_ready(sb));
+        warp_arrive(p_ready(sb), lane);
         continue;
       }
 
@@ -483,8 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           !(ok = warp_wait(pv_done(kept & 1), ((kept - 2) >> 1) & 1, abort_flag)))
         break;
       tmem_st_x64(lane_base + ((kept & 1) ? kColP1 : kColP0), pk);
-      tc_fence_before();
-      mbar_arrive(p_ready(sb));
+      warp_arrive(p_ready(sb), lane);
       ++kept;
     }
 
@@ -530,6 +534,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// Runs the kernels' bounded mbarrier wait on a barrier that nothing arrives
+// on, with a short limit: the wait must give up, raise the abort flag and
+// record the timeout in the status word, and the kernel must return.
+__global__ void wait_timeout_check_kernel(uint64_t limit_ns, int* result) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  mbar_init(smem_u32(&bar), 1);
+  fence_mbar_init();
+  const uint64_t t0 = globaltimer_ns();
+  const bool completed = wait_bar(smem_u32(&bar), 0, &abort_flag, limit_ns);
+  result[0] = completed ? 1 : 0;
+  result[1] = abort_flag;
+  result[2] = static_cast<int>((globaltimer_ns() - t0) / 1000);  // microseconds waited
 }
 
 // ----------------------------------------------------------------- host side
@@ -679,6 +700,13 @@ extern "C" int ssa_calibrate(const void* q, const void* k, const void* v, const 
 }
 
 extern "C" const char* ssa_last_cuda_error(void) { return t_last_cuda_error; }
+
+extern "C" int ssa_wait_timeout_check(int* result, int64_t limit_ns, void* stream) {
+  if (!result || limit_ns <= 0 || limit_ns > 1000000000) return SSA_ERR_INVALID_ARG;
+  wait_timeout_check_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_ns), result);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SSA_OK : cuda_fail(e);
+}
 
 extern "C" int ssa_get_error(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

@@ -140,6 +140,14 @@ int ssa_get_error(void* stream);
 /* Static description of a status code. */
 const char* ssa_status_string(int status);
 
+/* Diagnostic for failure detection: runs the kernels' bounded mbarrier wait
+ * (the one every producer/consumer wait uses) on a barrier nothing arrives
+ * on, giving up after limit_ns (1 .. 1e9). Writes device int[3]: completed
+ * (expected 0), abort flag raised (expected 1), microseconds waited. The
+ * wait also records SSA_ERR_TIMEOUT in the device status word, which
+ * ssa_get_error() then returns and clears. No fault, no hang. */
+int ssa_wait_timeout_check(int* result, int64_t limit_ns, void* stream);
+
 /* Text of the last CUDA error this library saw on the calling host thread
  * (the cause behind an SSA_ERR_CUDA); "no error" if none. Static storage. */
 const char* ssa_last_cuda_error(void);
