@@ -84,7 +84,7 @@ struct Ctl {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages];
   uint64_t s_full[2], p_ready[2], pv_done[2];  // pv_done[b] also frees V stage b
-  uint64_t dec_ready[kDecRing], s_free[2], drain;
+  uint64_t dec_ready[kDecRing], drain;
   uint32_t tmem_base;
   int abort_flag;
   int dec[kDecRing];
@@ -210,7 +210,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto p_ready = [&](int i) { return smem_u32(&ctl.p_ready[i]); };
   auto pv_done = [&](int i) { return smem_u32(&ctl.pv_done[i]); };
   auto dec_ready = [&](int i) { return smem_u32(&ctl.dec_ready[i]); };
-  auto s_free = [&](int i) { return smem_u32(&ctl.s_free[i]); };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -223,9 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full(i), 1);
-      mbar_init(p_ready(i), 4);  // one arrival per softmax warp
+      mbar_init(p_ready(i), 4);  // one arrival per softmax warp, per kept tile
       mbar_init(pv_done(i), 1);
-      mbar_init(s_free(i), 4);
     }
     for (int i = 0; i < kDecRing; ++i) mbar_init(dec_ready(i), 1);
     mbar_init(smem_u32(&ctl.drain), 1);
@@ -342,16 +340,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; ok && j < nkv; ++j) {
         const int t = j + 2;  // S_{j+2} goes to S_j's buffer
         if (MODE == kSkip) {
-          // Skipped tiles are short, so S_{j+2} is issued as soon as the
-          // softmax has loaded S_j, before waiting for P_j.
+          // The decision for tile j also says S_j has been read (all softmax
+          // warps loaded it before the vote's barrier): S_{j+2} is issued at
+          // once, and a skipped tile costs this thread no further wait.
+          if (!(ok = wait_bar(dec_ready(j % kDecRing), (j / kDecRing) & 1, abort_flag))) break;
+          const bool skip = reinterpret_cast<volatile int*>(ctl.dec)[j % kDecRing] != 0;
           if (t < nkv) {
-            if (!(ok = wait_bar(s_free(j & 1), (j >> 1) & 1, abort_flag))) break;
             if (!(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag))) break;
             tc_fence_after();
             issue_qk(t);
           }
-          if (!(ok = wait_bar(p_ready(j & 1), (j >> 1) & 1, abort_flag))) break;
-          if (reinterpret_cast<volatile int*>(ctl.dec)[j % kDecRing] != 0) continue;
+          if (skip) continue;
+          if (!(ok = wait_bar(p_ready(kept & 1), (kept >> 1) & 1, abort_flag))) break;
           const int vs = kept % kVStages;
           if (!(ok = wait_bar(v_full(vs), (kept / kVStages) & 1, abort_flag))) break;
           tc_fence_after();
@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // both groups back to back: tcgen05.mma issue is nearly synchronous,
           // so each wait on this thread is a tensor-pipe bubble. The softmax
           // finished reading S_j before arriving on p_ready for tile j.
-          if (!(ok = wait_bar(p_ready(j & 1), (j >> 1) & 1, abort_flag))) break;
+          if (!(ok = wait_bar(p_ready(kept & 1), (kept >> 1) & 1, abort_flag))) break;
           const int vs = kept % kVStages;
           if (!(ok = wait_bar(v_full(vs), (kept / kVStages) & 1, abort_flag))) break;
           if (t < nkv && !(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag))) break;
@@ -400,7 +400,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld_x128(lane_base + (sb ? kColS1 : kColS0), sr);
-      if (MODE == kSkip) warp_arrive(s_free(sb), lane);
       float s[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
@@ -412,17 +411,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float mx[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = s[i];
+      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(s[2 * i], s[2 * i + 1]);
 #pragma unroll
-      for (int i = 8; i < 128; ++i) mx[i & 7] = fmaxf(mx[i & 7], s[i]);
-      const float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
-                         c;
+      for (int i = 8; i < 64; ++i) mx[i & 7] = fmax3(mx[i & 7], s[2 * i], s[2 * i + 1]);
+      const float tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7])) * c;
 
       bool skip = false;
       if (MODE != kDense || EX) {
         const float dr = warp_max_f32(row_valid ? (tmax - m_true) : -INFINITY);
         if (lane == 0) ctl.red[sb][warp] = dr;
+        // S_j has been read into registers by every warp once this barrier
+        // completes: the decision barrier below then also frees S_j's buffer.
+        tc_fence_before();
         named_barrier_sync(kVoteBarrier, 128);
         volatile float* red = ctl.red[sb];
         const float d = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
@@ -443,9 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(dec_ready(j % kDecRing));
         }
       }
-      if (skip) {
+      if (skip) {  // nothing to hand over: P-ready counts kept tiles only
         ++nskip;
-        warp_arrive(p_ready(sb), lane);
         continue;
       }
 
@@ -488,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           !(ok = warp_wait(pv_done(kept & 1), ((kept - 2) >> 1) & 1, abort_flag)))
         break;
       tmem_st_x64(lane_base + ((kept & 1) ? kColP1 : kColP0), pk);
-      warp_arrive(p_ready(sb), lane);
+      warp_arrive(p_ready(kept & 1), lane);
       ++kept;
     }
 
