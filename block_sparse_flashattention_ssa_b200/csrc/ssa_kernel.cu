@@ -1,22 +1,32 @@
 // BLASST skip-softmax attention for B200 (sm_100a): forward with tile
 // skipping and the multi-threshold calibration pass.
 //
-// One CTA walks the KV tiles of one 128-row query block of one (sequence,
-// head). Warp roles:
-//   warp 4  TMA producer: Q once, K tiles through a 3-stage ring, and V tiles
-//           through a 2-stage ring -- V of tile j only once the softmax warps
-//           have decided to keep tile j (skipped tiles issue no V load);
-//   warp 5  tcgen05 issuer: once P_j is ready, O += P_j V_j (kept tiles only,
-//           P_j read from TMEM) and then S_{j+2} = Q K_{j+2}^T into the S
-//           buffer S_j has just freed (two TMEM S buffers, S two tiles ahead);
-//   warps 0-3  softmax, one query row per thread: row max of S_j in the log2
-//           domain, the CTA-wide skip vote d_j < log2(lambda) (Model-Optimizer
-//           commit page, "Triton kernels": tiles whose max score is far below
-//           the running max are skipped, no V load, softmax or accumulation),
-//           exponentials with a lazily rescaled reference max, P to TMEM, and
-//           the epilogue O / l -> bf16.
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O [256,256+D) P0 [384,448)
-// P1 [448,512), P stored as packed bf16 pairs.
+// One CTA takes two consecutive 128-row query blocks (X = A, B) of one
+// (sequence, head) and walks the sequence's KV tiles in order; both query
+// blocks share every K and V tile staged in shared memory. Warp roles:
+//   warps 0-3 / 4-7  softmax of query block A / B, one query row per thread:
+//           row max of S_X in the log2 domain, the block's skip vote
+//           d_j < log2(lambda) (Model-Optimizer commit page, "Triton kernels":
+//           tiles whose max score is far below the running max are skipped,
+//           no V load, softmax or accumulation), exponentials against a lazily
+//           rescaled reference max, P_X (bf16) written over S_X in TMEM, and
+//           the epilogue O_X / l -> bf16;
+//   warp 8  TMA producer: Q_A and Q_B once, K tiles through a 3-stage ring and
+//           V tiles through a 2-stage ring -- V_j only once A or B has decided
+//           to keep tile j (a tile both skip issues no V load);
+//   warp 9  tcgen05 issuer, per KV tile j and per block X in order A, B:
+//           O_X += P_X V_j (when X keeps j, P_X read from TMEM), then
+//           S_X = Q_X K_{j+1}^T into the same TMEM columns.
+// tcgen05 MMAs issued by one thread execute in issue order, so the S MMA
+// cannot overwrite P_X before the PV MMA ahead of it has read P_X; and a
+// commit tracks every earlier MMA of the thread, so when S_X(j+1) is reported
+// complete every MMA into O_X issued before it has completed too (the softmax
+// may rescale O_X and overwrite the P_X columns without a further wait).
+// The two softmax groups run out of phase: one group's exponentials overlap
+// the MMAs of the other.
+// TMEM (512 columns): S_A [0,128) S_B [128,256) O_A [256,256+D)
+// O_B [384,384+D); P_X occupies the first 64 columns of S_X as packed bf16
+// pairs.
 //
 // Every wait on an mbarrier is bounded in time; when one runs out the CTA
 // records SSA_ERR_TIMEOUT in the device status word, the other roles see the
@@ -38,22 +48,24 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kBM = SSA_TILE;  // query rows per tile
+constexpr int kBM = SSA_TILE;  // query rows per block
 constexpr int kBN = SSA_TILE;  // key/value rows per tile
-constexpr int kThreads = 192;
-constexpr int kTmaWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kQBlocks = 2;    // query blocks per CTA
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kThreads = 320;
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
-constexpr int kDecRing = 4;  // > kKStages - 1: bounds how far the vote runs ahead of the V producer
+constexpr int kDecRing = 4;  // > kKStages - 1: bounds how far a vote runs ahead of its readers
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP0 = 384, kColP1 = 448;
+__host__ __device__ constexpr uint32_t col_S(int x) { return x ? 128u : 0u; }    // S_X (and P_X)
+__host__ __device__ constexpr uint32_t col_O(int x) { return x ? 384u : 256u; }  // O_X
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 256 before a rescale
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kStatusTimeout = 1;
 constexpr int kStatusDeviceArg = 2;
 constexpr uint32_t kFull = 0xFFFFFFFFu;
-constexpr int kVoteBarrier = 1;  // named barrier of the four softmax warps (0 is __syncthreads)
+constexpr int kVoteBarrier = 1;  // named barriers 1 and 2: the vote of softmax group A and B
 
 enum Mode : int { kDense = 0, kSkip = 1, kCalib = 2 };
 
@@ -82,23 +94,24 @@ struct Params {
 struct Ctl {
   uint64_t bar_q;
   uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t v_full[kVStages];
-  uint64_t s_full[2], p_ready[2], pv_done[2];  // pv_done[b] also frees V stage b
-  uint64_t dec_ready[kDecRing], drain;
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[kQBlocks], p_ready[kQBlocks];
+  uint64_t dec_ready[kQBlocks][kDecRing];
+  uint64_t o_final, drain;
   uint32_t tmem_base;
   int abort_flag;
-  int dec[kDecRing];
-  float red[2][4];
-  int cnt[SSA_MAX_THRESHOLDS];  // calibration counts of this unit (thread 0 only)
-  int seq, qb, S, start, gqb, nq_total;
+  int dec[kQBlocks][kDecRing];
+  float red[kQBlocks][2][4];
+  int cnt[kQBlocks][SSA_MAX_THRESHOLDS];  // calibration counts of each block (its group's first thread)
+  int seq, qb_a, has_b, S, start, gqb_a, nq_total;
 };
 
 template <int D>
 struct Layout {
   static constexpr int kTileBytes = kBM * D * 2;  // 128 rows x D bf16, as D/64 chunks of 128 rows x 128 B
   static constexpr int kChunkBytes = kBM * 128;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
+  static constexpr int kQ = 0;  // Q_A, then Q_B
+  static constexpr int kK = kQ + kQBlocks * kTileBytes;
   static constexpr int kV = kK + kKStages * kTileBytes;
   static constexpr int kCtl = kV + kVStages * kTileBytes;
   static constexpr int kBytes = kCtl + static_cast<int>(sizeof(Ctl));
@@ -159,9 +172,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int head = blockIdx.y;
 
-  // Locate this CTA's (sequence, q-block) and validate cu_seqlens.
+  // Locate this CTA's (sequence, pair of q-blocks) and validate cu_seqlens.
   if (threadIdx.x == 0) {
-    int acc = 0, seq = -1, qb = 0, start = 0, S = 0, gqb = 0, bad = 0;
+    int accq = 0, accp = 0, seq = -1, qb_a = 0, has_b = 0, start = 0, S = 0, gqb_a = 0, bad = 0;
     int prev = p.cu_seqlens[0];
     if (prev < 0) bad = 1;
     for (int b = 0; b < p.batch && !bad; ++b) {
@@ -172,14 +185,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const int nq = (len + kBM - 1) / kBM;
-      if (seq < 0 && static_cast<int>(blockIdx.x) < acc + nq) {
+      const int np = (nq + 1) / 2;
+      if (seq < 0 && static_cast<int>(blockIdx.x) < accp + np) {
         seq = b;
-        qb = blockIdx.x - acc;
-        gqb = blockIdx.x;
+        qb_a = 2 * (static_cast<int>(blockIdx.x) - accp);
+        has_b = qb_a + 1 < nq ? 1 : 0;
+        gqb_a = accq + qb_a;
         start = prev;
         S = len;
       }
-      acc += nq;
+      accq += nq;
+      accp += np;
       prev = nxt;
     }
     if (!bad && seq >= 0 && (EX && (S + kBN - 1) / kBN > p.max_tiles)) bad = 1;
@@ -188,28 +204,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       seq = -1;
     }
     ctl.seq = seq;
-    ctl.qb = qb;
+    ctl.qb_a = qb_a;
+    ctl.has_b = has_b;
     ctl.S = S;
     ctl.start = start;
-    ctl.gqb = gqb;
-    ctl.nq_total = acc;
+    ctl.gqb_a = gqb_a;
+    ctl.nq_total = accq;
   }
   __syncthreads();
   if (ctl.seq < 0) return;  // uniform: no unit for this CTA (or bad input)
 
-  const int qb = ctl.qb, S = ctl.S, seq_start = ctl.start;
+  const int qb_a = ctl.qb_a, S = ctl.S, seq_start = ctl.start;
+  const int nx = ctl.has_b ? 2 : 1;  // query blocks this CTA holds
   const int nkv = (S + kBN - 1) / kBN;
-  const int64_t unit = static_cast<int64_t>(head) * ctl.nq_total + ctl.gqb;
   volatile int* abort_flag = &ctl.abort_flag;
 
   const uint32_t bar_q = smem_u32(&ctl.bar_q);
   auto k_full = [&](int i) { return smem_u32(&ctl.k_full[i]); };
   auto k_empty = [&](int i) { return smem_u32(&ctl.k_empty[i]); };
   auto v_full = [&](int i) { return smem_u32(&ctl.v_full[i]); };
-  auto s_full = [&](int i) { return smem_u32(&ctl.s_full[i]); };
-  auto p_ready = [&](int i) { return smem_u32(&ctl.p_ready[i]); };
-  auto pv_done = [&](int i) { return smem_u32(&ctl.pv_done[i]); };
-  auto dec_ready = [&](int i) { return smem_u32(&ctl.dec_ready[i]); };
+  auto v_empty = [&](int i) { return smem_u32(&ctl.v_empty[i]); };
+  auto s_full = [&](int x) { return smem_u32(&ctl.s_full[x]); };
+  auto p_ready = [&](int x) { return smem_u32(&ctl.p_ready[x]); };
+  auto dec_ready = [&](int x, int i) { return smem_u32(&ctl.dec_ready[x][i]); };
+  const uint32_t o_final = smem_u32(&ctl.o_final);
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
@@ -219,13 +237,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kVStages; ++i) {
       mbar_init(v_full(i), 1);
+      mbar_init(v_empty(i), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(s_full(i), 1);
-      mbar_init(p_ready(i), 4);  // one arrival per softmax warp, per kept tile
-      mbar_init(pv_done(i), 1);
+    for (int x = 0; x < kQBlocks; ++x) {
+      mbar_init(s_full(x), 1);
+      mbar_init(p_ready(x), 4);  // one arrival per softmax warp of the group, per kept tile
+      for (int i = 0; i < kDecRing; ++i) mbar_init(dec_ready(x, i), 1);
     }
-    for (int i = 0; i < kDecRing; ++i) mbar_init(dec_ready(i), 1);
+    mbar_init(o_final, 1);
     mbar_init(smem_u32(&ctl.drain), 1);
     ctl.abort_flag = 0;
     fence_mbar_init();
@@ -245,9 +264,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const uint32_t q_s = smem_u32(smem + L::kQ);
-      mbar_arrive_expect_tx(bar_q, L::kTileBytes);
-      for (int ch = 0; ch < D / 64; ++ch) tma_load_3d(q_s + ch * L::kChunkBytes, &tmQ, bar_q, ch * 64, head, seq_start + qb * kBM);
+      mbar_arrive_expect_tx(bar_q, nx * L::kTileBytes);
+      for (int x = 0; x < nx; ++x) {
+        const uint32_t q_s = smem_u32(smem + L::kQ + x * L::kTileBytes);
+        for (int ch = 0; ch < D / 64; ++ch)
+          tma_load_3d(q_s + ch * L::kChunkBytes, &tmQ, bar_q, ch * 64, head, seq_start + (qb_a + x) * kBM);
+      }
       int k_issued = 0, v_issued = 0;
       bool ok = true;
       for (int j = 0; j < nkv && ok; ++j) {
@@ -263,18 +285,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(dst + ch * L::kChunkBytes, &tmK, k_full(st), ch * 64, head, seq_start + k_issued * kBN);
         }
         if (!ok) break;
-        bool skip = false;
-        if (MODE == kSkip) {
-          if (!wait_bar(dec_ready(j % kDecRing), (j / kDecRing) & 1, abort_flag)) {
-            ok = false;
-            break;
+        bool need_v = true;
+        if (MODE == kSkip) {  // V_j is needed when either block keeps tile j
+          need_v = false;
+          for (int x = 0; x < nx && !need_v; ++x) {
+            if (!wait_bar(dec_ready(x, j % kDecRing), (j / kDecRing) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            need_v = reinterpret_cast<volatile int*>(ctl.dec[x])[j % kDecRing] == 0;
           }
-          skip = reinterpret_cast<volatile int*>(ctl.dec)[j % kDecRing] != 0;
+          if (!ok) break;
         }
-        if (!skip) {
+        if (need_v) {
           const int vs = v_issued % kVStages;
-          // V stage vs was last read by PV number v_issued - 2, which commits to pv_done[vs]
-          if (v_issued >= kVStages && !wait_bar(pv_done(vs), ((v_issued / kVStages) - 1) & 1, abort_flag)) {
+          if (v_issued >= kVStages && !wait_bar(v_empty(vs), ((v_issued / kVStages) - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -298,14 +323,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
-      const uint32_t q_s = smem_u32(smem + L::kQ);
-      // S_t = Q K_t^T into S buffer t & 1 (no waits inside: the caller has made
-      // sure K_t has landed and the buffer's previous S was consumed).
-      auto issue_qk = [&](int t) {
-        const int st = t % kKStages;
-        const int sb = t & 1;
-        const uint32_t k_s = smem_u32(smem + L::kK + st * L::kTileBytes);
-        const uint32_t d_tmem = tmem + (sb ? kColS1 : kColS0);
+      // S_X = Q_X K_t^T (the caller has made sure K_t has landed and that
+      // nothing still needs S_X's previous contents).
+      auto issue_qk = [&](int x, int t) {
+        const uint32_t q_s = smem_u32(smem + L::kQ + x * L::kTileBytes);
+        const uint32_t k_s = smem_u32(smem + L::kK + (t % kKStages) * L::kTileBytes);
+        const uint32_t d_tmem = tmem + col_S(x);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
           // K-major, 128B swizzle: 16-element k slices are 32 B apart inside a
@@ -314,74 +337,83 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(d_tmem, smem_desc_sw128(q_s + off, 16, 1024), smem_desc_sw128(k_s + off, 16, 1024), idesc_qk,
                  ks > 0 ? 1u : 0u);
         }
-        tc_commit(s_full(sb));
-        tc_commit(k_empty(st));
+        tc_commit(s_full(x));
       };
-      bool ok = wait_bar(bar_q, 0, abort_flag);
-      for (int t = 0; ok && t < 2 && t < nkv; ++t) {  // S_0 and S_1
-        if (!(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag))) break;
-        tc_fence_after();
-        issue_qk(t);
-      }
-      // O += P_j V_j from the TMEM copy of P_j and V stage vs.
-      auto issue_pv = [&](int kp, int vs) {
-        const uint32_t p_tmem = tmem + ((kp & 1) ? kColP1 : kColP0);
+      // O_X += P_X V from the TMEM copy of P_X and V stage vs.
+      auto issue_pv = [&](int x, int vs, bool accumulate) {
+        const uint32_t p_tmem = tmem + col_S(x);
         const uint32_t v_s = smem_u32(smem + L::kV + vs * L::kTileBytes);
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks) {
           // V is MN-major (d contiguous): 16 kv rows = 2 KB per k step; the
           // second 64-column chunk of d sits one 16 KB chunk further (LBO).
-          mma_ts(tmem + kColO, p_tmem + ks * 8, smem_desc_sw128(v_s + ks * 16 * 128, L::kChunkBytes, 1024),
-                 idesc_pv, (kp > 0 || ks > 0) ? 1u : 0u);
+          mma_ts(tmem + col_O(x), p_tmem + ks * 8, smem_desc_sw128(v_s + ks * 16 * 128, L::kChunkBytes, 1024),
+                 idesc_pv, (accumulate || ks > 0) ? 1u : 0u);
         }
-        tc_commit(pv_done(kp & 1));
       };
-      int kept = 0;
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int t = j + 2;  // S_{j+2} goes to S_j's buffer
-        if (MODE == kSkip) {
-          // The decision for tile j also says S_j has been read (all softmax
-          // warps loaded it before the vote's barrier): S_{j+2} is issued at
-          // once, and a skipped tile costs this thread no further wait.
-          if (!(ok = wait_bar(dec_ready(j % kDecRing), (j / kDecRing) & 1, abort_flag))) break;
-          const bool skip = reinterpret_cast<volatile int*>(ctl.dec)[j % kDecRing] != 0;
-          if (t < nkv) {
-            if (!(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag))) break;
-            tc_fence_after();
-            issue_qk(t);
-          }
-          if (skip) continue;
-          if (!(ok = wait_bar(p_ready(kept & 1), (kept >> 1) & 1, abort_flag))) break;
-          const int vs = kept % kVStages;
-          if (!(ok = wait_bar(v_full(vs), (kept / kVStages) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_pv(kept, vs);
-          ++kept;
-        } else {
-          // Wait once for everything O += P_j V_j and S_{j+2} need, then issue
-          // both groups back to back: tcgen05.mma issue is nearly synchronous,
-          // so each wait on this thread is a tensor-pipe bubble. The softmax
-          // finished reading S_j before arriving on p_ready for tile j.
-          if (!(ok = wait_bar(p_ready(kept & 1), (kept >> 1) & 1, abort_flag))) break;
-          const int vs = kept % kVStages;
-          if (!(ok = wait_bar(v_full(vs), (kept / kVStages) & 1, abort_flag))) break;
-          if (t < nkv && !(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_pv(kept, vs);
-          ++kept;
-          if (t < nkv) issue_qk(t);
-        }
+      bool ok = wait_bar(bar_q, 0, abort_flag) && wait_bar(k_full(0), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        for (int x = 0; x < nx; ++x) issue_qk(x, 0);
+        tc_commit(k_empty(0));
       }
-      if (!ok) {  // let every MMA issued so far finish before TMEM is released
+      int kept[kQBlocks] = {0, 0};
+      int v_used = 0;
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int t = j + 1;  // S_X(t) is issued right behind O_X += P_X(j) V_j
+        bool v_waited = false, k_waited = false;
+        for (int x = 0; x < nx; ++x) {
+          bool skip = false;
+          if (MODE == kSkip) {
+            // The decision also says every warp of the group has read S_X(j).
+            if (!(ok = wait_bar(dec_ready(x, j % kDecRing), (j / kDecRing) & 1, abort_flag))) break;
+            skip = reinterpret_cast<volatile int*>(ctl.dec[x])[j % kDecRing] != 0;
+          }
+          if (!skip) {
+            if (!(ok = wait_bar(p_ready(x), kept[x] & 1, abort_flag))) break;
+            if (!v_waited) {
+              if (!(ok = wait_bar(v_full(v_used % kVStages), (v_used / kVStages) & 1, abort_flag))) break;
+              v_waited = true;
+            }
+            tc_fence_after();
+            issue_pv(x, v_used % kVStages, kept[x] > 0);
+            ++kept[x];
+          }
+          if (t < nkv) {
+            if (!k_waited) {
+              if (!(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag))) break;
+              k_waited = true;
+            }
+            tc_fence_after();
+            issue_qk(x, t);
+          }
+        }
+        if (!ok) break;
+        if (v_waited) {  // V_j's stage is free once every PV on it has completed
+          tc_commit(v_empty(v_used % kVStages));
+          ++v_used;
+        }
+        if (t < nkv) tc_commit(k_empty(t % kKStages));
+      }
+      if (ok) {
+        tc_commit(o_final);
+      } else {  // let every MMA issued so far finish before TMEM is released
         tc_commit(smem_u32(&ctl.drain));
         drain_wait(smem_u32(&ctl.drain), 0);
       }
     }
-  } else {
+  } else if (warp < 4 * nx) {
     // ------------------------------------------------------------- softmax
-    const int row = warp * 32 + lane;
+    const int x = warp >> 2;   // query block of this warp's group
+    const int wq = warp & 3;   // TMEM lane quadrant = row group inside the block
+    const int gt = threadIdx.x & 127;  // thread index inside the group
+    const int qb = qb_a + x;
+    const int row = wq * 32 + lane;
     const bool row_valid = qb * kBM + row < S;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t col_s = col_S(x), col_o = col_O(x);
+    const int vote_bar = kVoteBarrier + x;
+    const int64_t unit = static_cast<int64_t>(head) * ctl.nq_total + ctl.gqb_a + x;
     const float c = p.c;
     float Lthr = -INFINITY;
     if (MODE == kSkip) Lthr = static_cast<float>(log2(static_cast<double>(p.tsf) / static_cast<double>(S)));
@@ -389,48 +421,61 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_used = -INFINITY;  // reference max of the exponentials (lags m_true by < kRescaleThreshold)
     float l = 0.f;
     int kept = 0, nskip = 0;
-    if (MODE == kCalib && threadIdx.x == 0)
-      for (int k = 0; k < SSA_MAX_THRESHOLDS; ++k) ctl.cnt[k] = 0;
+    if (MODE == kCalib && gt == 0)
+      for (int k = 0; k < SSA_MAX_THRESHOLDS; ++k) ctl.cnt[x][k] = 0;
     uint32_t bits = 0;
     bool ok = true;
 
     for (int j = 0; j < nkv; ++j) {
-      const int sb = j & 1;
-      if (!(ok = warp_wait(s_full(sb), (j >> 1) & 1, abort_flag))) break;
+      if (!(ok = warp_wait(s_full(x), j & 1, abort_flag))) break;
       tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld_x128(lane_base + (sb ? kColS1 : kColS0), sr);
-      float s[128];
-#pragma unroll
-      for (int i = 0; i < 128; ++i) s[i] = __uint_as_float(sr[i]);
-      const int valid = S - j * kBN;
-      if (valid < kBN) {
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i >= valid) s[i] = -INFINITY;
-      }
+      // S_X is read in two 64-column halves to bound register use: the upper
+      // half stays in registers, the lower half is read again for the
+      // exponentials of a kept tile.
+      const int valid = S - j * kBN;  // valid columns of this tile (masked to -inf past it)
       float mx[8];
+      {
+        uint32_t lo[64];
+        tmem_ld_x64(lane_base + col_s, lo);
+        if (valid < 64) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(s[2 * i], s[2 * i + 1]);
+          for (int i = 0; i < 64; ++i)
+            if (i >= valid) lo[i] = __float_as_uint(-INFINITY);
+        }
 #pragma unroll
-      for (int i = 8; i < 64; ++i) mx[i & 7] = fmax3(mx[i & 7], s[2 * i], s[2 * i + 1]);
+        for (int i = 0; i < 8; ++i) mx[i] = fmax3(__uint_as_float(lo[4 * i]), __uint_as_float(lo[4 * i + 1]),
+                                                   fmaxf(__uint_as_float(lo[4 * i + 2]), __uint_as_float(lo[4 * i + 3])));
+#pragma unroll
+        for (int i = 16; i < 32; ++i)
+          mx[i & 7] = fmax3(mx[i & 7], __uint_as_float(lo[2 * i]), __uint_as_float(lo[2 * i + 1]));
+      }
+      uint32_t hi[64];
+      tmem_ld_x64(lane_base + col_s + 64, hi);
+      if (valid < 128) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          if (64 + i >= valid) hi[i] = __float_as_uint(-INFINITY);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        mx[i & 7] = fmax3(mx[i & 7], __uint_as_float(hi[2 * i]), __uint_as_float(hi[2 * i + 1]));
       const float tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7])) * c;
 
       bool skip = false;
       if (MODE != kDense || EX) {
         const float dr = warp_max_f32(row_valid ? (tmax - m_true) : -INFINITY);
-        if (lane == 0) ctl.red[sb][warp] = dr;
-        // S_j has been read into registers by every warp once this barrier
-        // completes: the decision barrier below then also frees S_j's buffer.
+        if (lane == 0) ctl.red[x][j & 1][wq] = dr;
+        // S_X(j) has been read into registers by every warp of the group once
+        // this barrier completes: the decision below then also frees S_X.
         tc_fence_before();
-        named_barrier_sync(kVoteBarrier, 128);
-        volatile float* red = ctl.red[sb];
+        named_barrier_sync(vote_bar, 128);
+        volatile float* red = ctl.red[x][j & 1];
         const float d = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
         if (MODE == kSkip) skip = d < Lthr;
-        if (MODE == kCalib && threadIdx.x == 0) {
-          for (int k = 0; k < p.n_cal; ++k) ctl.cnt[k] += d < p.Lcal[k] ? 1 : 0;
+        if (MODE == kCalib && gt == 0) {
+          for (int k = 0; k < p.n_cal; ++k) ctl.cnt[x][k] += d < p.Lcal[k] ? 1 : 0;
         }
-        if (EX && threadIdx.x == 0) {
+        if (EX && gt == 0) {
           if (p.tile_stat) p.tile_stat[unit * p.max_tiles + j] = d;
           bits |= (skip ? 1u : 0u) << (j & 31);
           if ((j & 31) == 31 || j == nkv - 1) {
@@ -438,9 +483,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             bits = 0;
           }
         }
-        if (MODE == kSkip && threadIdx.x == 0) {
-          reinterpret_cast<volatile int*>(ctl.dec)[j % kDecRing] = skip ? 1 : 0;
-          mbar_arrive(dec_ready(j % kDecRing));
+        if (MODE == kSkip && gt == 0) {
+          reinterpret_cast<volatile int*>(ctl.dec[x])[j % kDecRing] = skip ? 1 : 0;
+          mbar_arrive(dec_ready(x, j % kDecRing));
         }
       }
       if (skip) {  // nothing to hand over: P-ready counts kept tiles only
@@ -448,7 +493,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         continue;
       }
 
-      // Kept tile: online softmax update.
+      // Kept tile: online softmax update. Every earlier MMA into O_X has
+      // completed (S_X(j) completing implies it), so O_X may be rescaled here.
       const float m_new = fmaxf(m_true, tmax);
       m_true = m_new;
       float alpha = 1.f;
@@ -456,48 +502,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         alpha = ex2_approx(m_used - m_new);  // 0 before the first kept tile
         m_used = m_new;
         if (kept > 0) {
-          if (!(ok = warp_wait(pv_done((kept - 1) & 1), ((kept - 1) >> 1) & 1, abort_flag))) break;
-          tc_fence_after();
 #pragma unroll
           for (int ch = 0; ch < D / 32; ++ch) {
             uint32_t o[32];
-            tmem_ld_x32(lane_base + kColO + ch * 32, o);
+            tmem_ld_x32(lane_base + col_o + ch * 32, o);
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st_x32(lane_base + kColO + ch * 32, o);
+            tmem_st_x32(lane_base + col_o + ch * 32, o);
           }
         }
       }
       l *= alpha;
       const float neg_m = -m_used;
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[64];
+      uint32_t pk_hi[32];  // P columns [64,128) -> packed TMEM columns [32,64)
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2_approx(fmaf(s[2 * i], c, neg_m));
-        const float p1 = ex2_approx(fmaf(s[2 * i + 1], c, neg_m));
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = ex2_approx(fmaf(__uint_as_float(hi[2 * i]), c, neg_m));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(hi[2 * i + 1]), c, neg_m));
         rs[i & 3] += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
+        pk_hi[i] = pack_bf16x2(p0, p1);
       }
+      {
+        uint32_t lo[64];
+        tmem_ld_x64(lane_base + col_s, lo);
+        if (valid < 64) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            if (i >= valid) lo[i] = __float_as_uint(-INFINITY);
+        }
+        uint32_t pk_lo[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(lo[2 * i]), c, neg_m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(lo[2 * i + 1]), c, neg_m));
+          rs[i & 3] += p0 + p1;
+          pk_lo[i] = pack_bf16x2(p0, p1);
+        }
+        // Both halves of S_X are in registers by now: P_X may overwrite them.
+        tmem_st_x32(lane_base + col_s, pk_lo);
+      }
+      tmem_st_x32(lane_base + col_s + 32, pk_hi);
       l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-      // P buffer kept & 1 was last read by the PV two kept tiles back. In the
-      // dense and calibration order that PV was issued before S_j and so
-      // completed before S_j did; in skip mode S is issued ahead of PV, so wait.
-      if (MODE == kSkip && kept >= 2 &&
-          !(ok = warp_wait(pv_done(kept & 1), ((kept - 2) >> 1) & 1, abort_flag)))
-        break;
-      tmem_st_x64(lane_base + ((kept & 1) ? kColP1 : kColP0), pk);
-      warp_arrive(p_ready(kept & 1), lane);
+      warp_arrive(p_ready(x), lane);
       ++kept;
     }
 
-    // A warp that left the loop on an error arrives once on the vote barrier,
-    // so the other softmax warps cannot be left waiting at it: the barrier is
-    // a full barrier per tile, so no warp is ever more than one instance away.
-    if (!ok && (MODE != kDense || EX)) named_barrier_arrive(kVoteBarrier, 128);
+    // A warp that left the loop on an error arrives once on its group's vote
+    // barrier, so the group's other warps cannot be left waiting at it: the
+    // barrier is a full barrier per tile, so no warp is more than one instance away.
+    if (!ok && (MODE != kDense || EX)) named_barrier_arrive(vote_bar, 128);
 
-    // Epilogue: O / l -> bf16, masked row stores; per-unit counters.
-    if (ok && kept > 0) ok = warp_wait(pv_done((kept - 1) & 1), ((kept - 1) >> 1) & 1, abort_flag);
+    // Epilogue: O_X / l -> bf16, masked row stores; per-unit counters.
+    if (ok) ok = warp_wait(o_final, 0, abort_flag);
     if (ok) {
       tc_fence_after();
       const float inv_l = 1.0f / l;
@@ -506,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t o[32];
-        tmem_ld_x32(lane_base + kColO + ch * 32, o);
+        tmem_ld_x32(lane_base + col_o + ch * 32, o);
         uint32_t w[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -517,10 +574,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (threadIdx.x == 0) {
+      if (gt == 0) {
         if (p.skip_counter) p.skip_counter[unit] = nskip;
         if (MODE == kCalib) {
-          for (int k = 0; k < p.n_cal; ++k) p.counts[unit * p.n_cal + k] = ctl.cnt[k];
+          for (int k = 0; k < p.n_cal; ++k) p.counts[unit * p.n_cal + k] = ctl.cnt[x][k];
         }
       }
     }
@@ -630,8 +687,9 @@ int launch(const Call& a, const Params& p) {
   constexpr int smem = Layout<D>::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e);
-  // one CTA per query block: sum over sequences of ceil(S_b / 128) <= ceil(T / 128) + batch
-  const dim3 grid(static_cast<unsigned>((a.total_tokens + kBM - 1) / kBM + a.batch), static_cast<unsigned>(a.H));
+  // one CTA per pair of query blocks: sum over sequences of ceil(S_b / 256) <= ceil(T / 256) + batch
+  const dim3 grid(static_cast<unsigned>((a.total_tokens + 2 * kBM - 1) / (2 * kBM) + a.batch),
+                  static_cast<unsigned>(a.H));
   kernel<<<grid, kThreads, smem, a.stream>>>(tq, tk, tv, p);
   e = cudaGetLastError();
   return e == cudaSuccess ? SSA_OK : cuda_fail(e);
