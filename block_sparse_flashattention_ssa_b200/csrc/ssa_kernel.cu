@@ -429,36 +429,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < nkv; ++j) {
       if (!(ok = warp_wait(s_full(x), j & 1, abort_flag))) break;
       tc_fence_after();
-      // S_X is read in two 64-column halves to bound register use: the upper
-      // half stays in registers, the lower half is read again for the
-      // exponentials of a kept tile.
+      // S_X is read whole for the row max; only its upper 64 columns stay in
+      // registers, the lower half is read again (asynchronously) for the
+      // exponentials of a kept tile, to bound register use.
       const int valid = S - j * kBN;  // valid columns of this tile (masked to -inf past it)
+      uint32_t hi[64];
       float mx[8];
       {
-        uint32_t lo[64];
-        tmem_ld_x64(lane_base + col_s, lo);
-        if (valid < 64) {
+        uint32_t sr[128];
+        tmem_ld_x128(lane_base + col_s, sr);
+        if (valid < kBN) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (i >= valid) lo[i] = __float_as_uint(-INFINITY);
+          for (int i = 0; i < 128; ++i)
+            if (i >= valid) sr[i] = __float_as_uint(-INFINITY);
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmax3(__uint_as_float(lo[4 * i]), __uint_as_float(lo[4 * i + 1]),
-                                                   fmaxf(__uint_as_float(lo[4 * i + 2]), __uint_as_float(lo[4 * i + 3])));
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
 #pragma unroll
-        for (int i = 16; i < 32; ++i)
-          mx[i & 7] = fmax3(mx[i & 7], __uint_as_float(lo[2 * i]), __uint_as_float(lo[2 * i + 1]));
+        for (int i = 8; i < 64; ++i)
+          mx[i & 7] = fmax3(mx[i & 7], __uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1]));
+#pragma unroll
+        for (int i = 0; i < 64; ++i) hi[i] = sr[64 + i];
       }
-      uint32_t hi[64];
-      tmem_ld_x64(lane_base + col_s + 64, hi);
-      if (valid < 128) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (64 + i >= valid) hi[i] = __float_as_uint(-INFINITY);
-      }
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        mx[i & 7] = fmax3(mx[i & 7], __uint_as_float(hi[2 * i]), __uint_as_float(hi[2 * i + 1]));
       const float tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7])) * c;
 
       bool skip = false;
@@ -513,37 +505,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       l *= alpha;
-      const float neg_m = -m_used;
-      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_used, -m_used);
+      float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      uint32_t lo[64];
+      tmem_ld_x64_async(lane_base + col_s, lo);  // lands while the upper half is exponentiated
       uint32_t pk_hi[32];  // P columns [64,128) -> packed TMEM columns [32,64)
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(hi[2 * i]), c, neg_m));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(hi[2 * i + 1]), c, neg_m));
-        rs[i & 3] += p0 + p1;
-        pk_hi[i] = pack_bf16x2(p0, p1);
+        const float2 a = ffma2(make_float2(__uint_as_float(hi[2 * i]), __uint_as_float(hi[2 * i + 1])), c2, nm2);
+        const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+        rs[i & 1] = fadd2(rs[i & 1], e);
+        pk_hi[i] = pack_bf16x2(e.x, e.y);
       }
-      {
-        uint32_t lo[64];
-        tmem_ld_x64(lane_base + col_s, lo);
-        if (valid < 64) {
+      tmem_wait_ld_tied(lo);
+      if (valid < 64) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (i >= valid) lo[i] = __float_as_uint(-INFINITY);
-        }
-        uint32_t pk_lo[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(lo[2 * i]), c, neg_m));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(lo[2 * i + 1]), c, neg_m));
-          rs[i & 3] += p0 + p1;
-          pk_lo[i] = pack_bf16x2(p0, p1);
-        }
-        // Both halves of S_X are in registers by now: P_X may overwrite them.
-        tmem_st_x32(lane_base + col_s, pk_lo);
+        for (int i = 0; i < 64; ++i)
+          if (i >= valid) lo[i] = __float_as_uint(-INFINITY);
       }
+      uint32_t pk_lo[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float2 a = ffma2(make_float2(__uint_as_float(lo[2 * i]), __uint_as_float(lo[2 * i + 1])), c2, nm2);
+        const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+        rs[i & 1] = fadd2(rs[i & 1], e);
+        pk_lo[i] = pack_bf16x2(e.x, e.y);
+      }
+      // Both halves of S_X are in registers by now: P_X may overwrite them.
+      tmem_st_x32(lane_base + col_s, pk_lo);
       tmem_st_x32(lane_base + col_s + 32, pk_hi);
-      l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+      l += (rs[0].x + rs[1].x) + (rs[0].y + rs[1].y);
       warp_arrive(p_ready(x), lane);
       ++kept;
     }
