@@ -175,24 +175,24 @@ def weak_scaling_value(flop_per_rank: float, world: int, max_ms: float) -> float
 # --------------------------------------------------------------- our arm
 
 def calibrate_and_fit(ssa, dq, dk, dv, dcu, w):
-    import synth
-
-    lams = synth.CALIB_THRESHOLDS
+    """Count with ssa_calibrate (timed), then one fit point per (sequence,
+    trial) and the log-space fit (block_sparse_flashattention_ssa_b200.calibration)."""
     import torch
 
+    from block_sparse_flashattention_ssa_b200 import calibration as cal
+
+    lams = cal.DEFAULT_TRIALS
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
-    _, counts = ssa.calibrate(dq, dk, dv, dcu, w.max_seqlen, lams)
+    _, counts = ssa.calibrate(dq, dk, dv, dcu, w.max_seqlen, list(lams))
     e1.record()
     ssa.check_device()
     calib_ms = e0.elapsed_time(e1)
-    tiles = tiles_of(w.seqlens, w.H)
-    sparsity = counts.sum(dim=(0, 1)).double().cpu().numpy() / tiles
-    S = w.seqlens[0]
-    a, b, smin, smax = ssa.fit_logspace(sparsity, [lam * S for lam in lams])
-    return dict(a=a, b=b, s_min=smin, s_max=smax, calib_ms=calib_ms,
-                points=[[float(s), float(l)] for s, l in zip(sparsity, lams)])
+    seq = cal.sequence_counts(counts.cpu().numpy(), w.cu_seqlens)
+    c = cal.fit(cal.fit_points(seq, w.cu_seqlens, lams, total_heads=w.H))
+    return dict(a=c.a, b=c.b, s_min=c.s_min, s_max=c.s_max, calib_ms=calib_ms,
+                points=[[float(s), float(sf)] for s, sf in c.points])
 
 
 def time_fwd(ssa, args_fn, reps, stream):
