@@ -9,6 +9,8 @@ fails loudly when the library is missing.
 Entry points (same names as the C ABI, without the ``ssa_`` prefix):
   fwd          skip-softmax attention forward (optionally with per-tile
                diagnostics, the ``ssa_fwd_ex`` call)
+  fwd_fp8      the forward with E4M3 Q and K (per-tensor descales)
+  quantize_fp8 bf16 -> E4M3 per-tensor quantisation for fwd_fp8
   calibrate    dense attention + skip counts at N thresholds at once
   resolve      threshold_scale_factor = a * exp(b * target_sparsity)
   fit_logspace log-space least-squares fit of (a, b)
@@ -54,6 +56,10 @@ def _load():
     L.ssa_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp]
     L.ssa_fwd_ex.restype = i32
     L.ssa_fwd_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp, vp, vp]
+    L.ssa_fwd_fp8.restype = i32
+    L.ssa_fwd_fp8.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32, f32, vp, vp, vp, vp, vp]
+    L.ssa_quantize_fp8.restype = i32
+    L.ssa_quantize_fp8.argtypes = [vp, vp, ctypes.c_int64, f32, vp]
     L.ssa_calibrate.restype = i32
     L.ssa_calibrate.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32, vp, vp, vp]
     L.ssa_resolve.restype = f64
@@ -139,6 +145,36 @@ def fwd(q, k, v, cu_seqlens, max_seqlen: int, threshold_scale_factor: float = 0.
         _check(rc, "ssa_fwd_ex")
     else:
         _check(_lib.ssa_fwd(*args, _stream_handle(stream)), "ssa_fwd")
+    return out
+
+
+def fwd_fp8(q8, k8, v, cu_seqlens, max_seqlen: int, q_descale: float, k_descale: float,
+            threshold_scale_factor: float = 0.0, softmax_scale: float = 0.0, out=None, skip_counter=None,
+            decision_bitmap=None, tile_stat=None, stream=None):
+    """Forward with E4M3 Q and K (CUDA uint8 [total_tokens, H, 128], values
+    q_descale * decode(q8)) and bf16 V; returns bf16 ``out``."""
+    import torch
+
+    total, H, D = _shape(q8)
+    if out is None:
+        out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    batch = cu_seqlens.numel() - 1
+    rc = _lib.ssa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D,
+                          float(softmax_scale), float(q_descale), float(k_descale), float(threshold_scale_factor),
+                          _ptr(out), _ptr(skip_counter), _ptr(decision_bitmap), _ptr(tile_stat),
+                          _stream_handle(stream))
+    _check(rc, "ssa_fwd_fp8")
+    return out
+
+
+def quantize_fp8(x, inv_scale: float, out=None, stream=None):
+    """E4M3 codes (uint8, same shape) of fp32(x * inv_scale), nearest even, saturating."""
+    import torch
+
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(_lib.ssa_quantize_fp8(_ptr(x), _ptr(out), x.numel(), float(inv_scale), _stream_handle(stream)),
+           "ssa_quantize_fp8")
     return out
 
 

@@ -106,14 +106,20 @@ struct Ctl {
   int seq, qb_a, has_b, S, start, gqb_a, nq_total;
 };
 
-template <int D>
+// Shared-memory layout. Q and K are bf16, or E4M3 bytes when F8; V is bf16.
+// Every tile is stored as chunks of 128 rows x 128 B with the 128-byte swizzle.
+template <int D, bool F8>
 struct Layout {
-  static constexpr int kTileBytes = kBM * D * 2;  // 128 rows x D bf16, as D/64 chunks of 128 rows x 128 B
+  static constexpr int kQKElem = F8 ? 1 : 2;                  // bytes per Q/K element
+  static constexpr int kQKTileBytes = kBM * D * kQKElem;
+  static constexpr int kQKChunkElems = 128 / kQKElem;         // Q/K elements per 128-B row of a chunk
+  static constexpr int kQKChunks = D / kQKChunkElems;
+  static constexpr int kVTileBytes = kBN * D * 2;
   static constexpr int kChunkBytes = kBM * 128;
   static constexpr int kQ = 0;  // Q_A, then Q_B
-  static constexpr int kK = kQ + kQBlocks * kTileBytes;
-  static constexpr int kV = kK + kKStages * kTileBytes;
-  static constexpr int kCtl = kV + kVStages * kTileBytes;
+  static constexpr int kK = kQ + kQBlocks * kQKTileBytes;
+  static constexpr int kV = kK + kKStages * kQKTileBytes;
+  static constexpr int kCtl = kV + kVStages * kVTileBytes;
   static constexpr int kBytes = kCtl + static_cast<int>(sizeof(Ctl));
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B (128B swizzle atoms)
 };
@@ -160,11 +166,11 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-template <int D, int MODE, bool EX>
+template <int D, int MODE, bool EX, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     ssa_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params p) {
-  using L = Layout<D>;
+  using L = Layout<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl& ctl = *reinterpret_cast<Ctl*>(smem + L::kCtl);
@@ -264,11 +270,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      mbar_arrive_expect_tx(bar_q, nx * L::kTileBytes);
+      mbar_arrive_expect_tx(bar_q, nx * L::kQKTileBytes);
       for (int x = 0; x < nx; ++x) {
-        const uint32_t q_s = smem_u32(smem + L::kQ + x * L::kTileBytes);
-        for (int ch = 0; ch < D / 64; ++ch)
-          tma_load_3d(q_s + ch * L::kChunkBytes, &tmQ, bar_q, ch * 64, head, seq_start + (qb_a + x) * kBM);
+        const uint32_t q_s = smem_u32(smem + L::kQ + x * L::kQKTileBytes);
+        for (int ch = 0; ch < L::kQKChunks; ++ch)
+          tma_load_3d(q_s + ch * L::kChunkBytes, &tmQ, bar_q, ch * L::kQKChunkElems, head,
+                      seq_start + (qb_a + x) * kBM);
       }
       int k_issued = 0, v_issued = 0;
       bool ok = true;
@@ -279,10 +286,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const uint32_t dst = smem_u32(smem + L::kK + st * L::kTileBytes);
-          mbar_arrive_expect_tx(k_full(st), L::kTileBytes);
-          for (int ch = 0; ch < D / 64; ++ch)
-            tma_load_3d(dst + ch * L::kChunkBytes, &tmK, k_full(st), ch * 64, head, seq_start + k_issued * kBN);
+          const uint32_t dst = smem_u32(smem + L::kK + st * L::kQKTileBytes);
+          mbar_arrive_expect_tx(k_full(st), L::kQKTileBytes);
+          for (int ch = 0; ch < L::kQKChunks; ++ch)
+            tma_load_3d(dst + ch * L::kChunkBytes, &tmK, k_full(st), ch * L::kQKChunkElems, head,
+                        seq_start + k_issued * kBN);
         }
         if (!ok) break;
         bool need_v = true;
@@ -303,8 +311,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          const uint32_t dst = smem_u32(smem + L::kV + vs * L::kTileBytes);
-          mbar_arrive_expect_tx(v_full(vs), L::kTileBytes);
+          const uint32_t dst = smem_u32(smem + L::kV + vs * L::kVTileBytes);
+          mbar_arrive_expect_tx(v_full(vs), L::kVTileBytes);
           for (int ch = 0; ch < D / 64; ++ch)
             tma_load_3d(dst + ch * L::kChunkBytes, &tmV, v_full(vs), ch * 64, head, seq_start + j * kBN);
           ++v_issued;
@@ -321,28 +329,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------- tcgen05 issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_f32(kBM, kBN) : idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
       // S_X = Q_X K_t^T (the caller has made sure K_t has landed and that
       // nothing still needs S_X's previous contents).
       auto issue_qk = [&](int x, int t) {
-        const uint32_t q_s = smem_u32(smem + L::kQ + x * L::kTileBytes);
-        const uint32_t k_s = smem_u32(smem + L::kK + (t % kKStages) * L::kTileBytes);
+        const uint32_t q_s = smem_u32(smem + L::kQ + x * L::kQKTileBytes);
+        const uint32_t k_s = smem_u32(smem + L::kK + (t % kKStages) * L::kQKTileBytes);
         const uint32_t d_tmem = tmem + col_S(x);
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          // K-major, 128B swizzle: 16-element k slices are 32 B apart inside a
-          // 128-B row; every 64 elements start a new 16 KB chunk.
+        for (int ks = 0; ks < D * L::kQKElem / 32; ++ks) {
+          // K-major, 128B swizzle: each MMA takes 32 B of K (16 bf16 or 32
+          // E4M3 elements), 32 B apart inside a 128-B row; every 128 B of a
+          // row start a new 16 KB chunk.
           const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
-          mma_ss(d_tmem, smem_desc_sw128(q_s + off, 16, 1024), smem_desc_sw128(k_s + off, 16, 1024), idesc_qk,
-                 ks > 0 ? 1u : 0u);
+          const uint64_t da = smem_desc_sw128(q_s + off, 16, 1024), db = smem_desc_sw128(k_s + off, 16, 1024);
+          if (F8)
+            mma_ss_f8(d_tmem, da, db, idesc_qk, ks > 0 ? 1u : 0u);
+          else
+            mma_ss(d_tmem, da, db, idesc_qk, ks > 0 ? 1u : 0u);
         }
         tc_commit(s_full(x));
       };
       // O_X += P_X V from the TMEM copy of P_X and V stage vs.
       auto issue_pv = [&](int x, int vs, bool accumulate) {
         const uint32_t p_tmem = tmem + col_S(x);
-        const uint32_t v_s = smem_u32(smem + L::kV + vs * L::kTileBytes);
+        const uint32_t v_s = smem_u32(smem + L::kV + vs * L::kVTileBytes);
 #pragma unroll
         for (int ks = 0; ks < kBN / 16; ++ks) {
           // V is MN-major (d contiguous): 16 kv rows = 2 KB per k step; the
@@ -614,18 +626,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [total_tokens, H, D] bf16 viewed as a 3-D tensor (d, head, token); box of
-// 64 d x 1 head x 128 tokens with 128-byte swizzle. Rows past total_tokens
-// read as zero.
-bool make_tensor_map(CUtensorMap* map, const void* base, int total_tokens, int H, int D) {
+// [total_tokens, H, D] viewed as a 3-D tensor (d, head, token) of bf16 (or
+// of bytes, for E4M3); box of 128 bytes of d x 1 head x 128 tokens with
+// 128-byte swizzle. Rows past total_tokens read as zero.
+bool make_tensor_map(CUtensorMap* map, const void* base, int total_tokens, int H, int D, bool bytes) {
   auto encode = encode_fn();
   if (!encode) return false;
+  const cuuint64_t esize = bytes ? 1 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(total_tokens)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
-  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(kBN)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * esize, static_cast<cuuint64_t>(H) * D * esize};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esize), 1, static_cast<cuuint32_t>(kBN)};
   cuuint32_t estr[3] = {1, 1, 1};
-  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return encode(map, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -636,6 +650,8 @@ struct Call {
   float softmax_scale;
   void* out;
   cudaStream_t stream;
+  bool f8 = false;              // Q and K are E4M3 bytes
+  double qk_descale = 1.0;      // q_descale * k_descale (E4M3 only)
 };
 
 // Host-side argument check. total_tokens == 0 is a valid no-op whatever the
@@ -645,6 +661,8 @@ int validate(const Call& a) {
     return SSA_ERR_INVALID_ARG;
   if (std::isnan(a.softmax_scale) || std::isinf(a.softmax_scale)) return SSA_ERR_INVALID_ARG;
   if (a.D != 64 && a.D != 128) return SSA_ERR_UNSUPPORTED;
+  if (a.f8 && a.D != 128) return SSA_ERR_UNSUPPORTED;  // E4M3 rows of 128 B: one swizzle atom per row
+  if (a.f8 && !(a.qk_descale > 0.0 && std::isfinite(a.qk_descale))) return SSA_ERR_INVALID_ARG;
   if (a.total_tokens == 0) return SSA_OK;
   if (!a.q || !a.k || !a.v || !a.out) return SSA_ERR_INVALID_ARG;
   for (const void* ptr : {a.q, a.k, a.v, static_cast<const void*>(a.out)})
@@ -661,21 +679,22 @@ Params base_params(const Call& a) {
   p.num_heads = a.H;
   p.max_tiles = (a.max_seqlen + kBN - 1) / kBN;
   p.bitmap_words = (p.max_tiles + 31) / 32;
-  const double scale = a.softmax_scale > 0.f ? static_cast<double>(a.softmax_scale) : 1.0 / std::sqrt(static_cast<double>(a.D));
+  double scale = a.softmax_scale > 0.f ? static_cast<double>(a.softmax_scale) : 1.0 / std::sqrt(static_cast<double>(a.D));
+  if (a.f8) scale = scale * a.qk_descale;  // E4M3 codes carry the per-tensor scales of Q and K
   p.c = static_cast<float>(scale * 1.4426950408889634073599246810019);
   return p;
 }
 
-template <int D, int MODE, bool EX>
+template <int D, int MODE, bool EX, bool F8>
 int launch(const Call& a, const Params& p) {
   CUtensorMap tq, tk, tv;
-  if (!make_tensor_map(&tq, a.q, a.total_tokens, a.H, D) || !make_tensor_map(&tk, a.k, a.total_tokens, a.H, D) ||
-      !make_tensor_map(&tv, a.v, a.total_tokens, a.H, D)) {
+  if (!make_tensor_map(&tq, a.q, a.total_tokens, a.H, D, F8) || !make_tensor_map(&tk, a.k, a.total_tokens, a.H, D, F8) ||
+      !make_tensor_map(&tv, a.v, a.total_tokens, a.H, D, false)) {
     t_last_cuda_error = "cuTensorMapEncodeTiled failed or the driver entry point is unavailable";
     return SSA_ERR_CUDA;
   }
-  auto kernel = ssa_attention_kernel<D, MODE, EX>;
-  constexpr int smem = Layout<D>::kAlloc;
+  auto kernel = ssa_attention_kernel<D, MODE, EX, F8>;
+  constexpr int smem = Layout<D, F8>::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e);
   // one CTA per pair of query blocks: sum over sequences of ceil(S_b / 256) <= ceil(T / 256) + batch
@@ -688,7 +707,39 @@ int launch(const Call& a, const Params& p) {
 
 template <int MODE, bool EX>
 int dispatch_d(const Call& a, const Params& p) {
-  return a.D == 64 ? launch<64, MODE, EX>(a, p) : launch<128, MODE, EX>(a, p);
+  if (a.f8) return launch<128, MODE, EX, true>(a, p);
+  return a.D == 64 ? launch<64, MODE, EX, false>(a, p) : launch<128, MODE, EX, false>(a, p);
+}
+
+// y = E4M3(fp32(x * inv_scale)), round to nearest even, saturating to +-448;
+// eight elements per thread (16-byte loads, 8-byte stores), a scalar tail.
+__global__ void quantize_e4m3_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ y, int64_t n,
+                                     float inv_scale) {
+  auto cvt2 = [](float lo, float hi) -> uint32_t {
+    unsigned short r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+  };
+  const int64_t groups = n / 8;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < groups; g += stride) {
+    const uint4 v = reinterpret_cast<const uint4*>(x)[g];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[2] = {0, 0};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float lo = __uint_as_float(w[i] << 16) * inv_scale;
+      const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * inv_scale;
+      o[i >> 1] |= cvt2(lo, hi) << ((i & 1) * 16);
+    }
+    reinterpret_cast<uint2*>(y)[g] = make_uint2(o[0], o[1]);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    for (int64_t i = groups * 8; i < n; ++i) {
+      const float f = __bfloat162float(x[i]) * inv_scale;
+      y[i] = static_cast<uint8_t>(cvt2(f, 0.f) & 0xFFu);
+    }
+  }
 }
 
 int fwd_impl(const Call& a, float tsf, int32_t* skip_counter, uint32_t* bitmap, float* tile_stat) {
@@ -711,6 +762,34 @@ int fwd_impl(const Call& a, float tsf, int32_t* skip_counter, uint32_t* bitmap, 
 }  // namespace ssa
 
 using namespace ssa;
+
+extern "C" int ssa_fwd_fp8(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                           int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                           float q_descale, float k_descale, float threshold_scale_factor, void* out,
+                           int32_t* skip_counter, uint32_t* decision_bitmap, float* tile_stat, void* stream) {
+  Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
+         static_cast<cudaStream_t>(stream)};
+  if (!(q_descale > 0.f) || !(k_descale > 0.f) || std::isinf(q_descale) || std::isinf(k_descale))
+    return SSA_ERR_INVALID_ARG;
+  a.f8 = true;
+  a.qk_descale = static_cast<double>(q_descale) * static_cast<double>(k_descale);
+  return fwd_impl(a, threshold_scale_factor, skip_counter, decision_bitmap, tile_stat);
+}
+
+extern "C" int ssa_quantize_fp8(const void* x, void* y, int64_t n, float inv_scale, void* stream) {
+  if (n < 0 || !(inv_scale > 0.f) || std::isinf(inv_scale)) return SSA_ERR_INVALID_ARG;
+  if (n == 0) return SSA_OK;
+  if (!x || !y) return SSA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(y) & 7u)) return SSA_ERR_UNSUPPORTED;
+  const int64_t groups = n / 8;
+  const int threads = 256;
+  const int64_t want = (groups + threads - 1) / threads;
+  const unsigned blocks = static_cast<unsigned>(want < 1 ? 1 : (want > 148 * 16 ? 148 * 16 : want));
+  quantize_e4m3_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<uint8_t*>(y), n, inv_scale);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? SSA_OK : cuda_fail(e);
+}
 
 extern "C" int ssa_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
                        int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,

@@ -110,6 +110,37 @@ int ssa_calibrate(const void* q, const void* k, const void* v, const int32_t* cu
                   const float* thresholds, int n_thresholds, void* out, int32_t* counts, void* stream);
 
 /*
+ * ssa_fwd_ex with 8-bit Q and K: S = Q K^T runs on E4M3 operands (OCP FP8,
+ * no infinities; tcgen05 kind::f8f6f4) while V, P and the output stay bf16.
+ * The TRT-LLM docs ("VisualGen Sparse Attention (Beta)", "User
+ * Configuration") state that skip-softmax composes with quantised Q/K
+ * attention; its pull-request page ("Benchmark") reports FP8 speed-ups.
+ * Reading: one scale per tensor, so the real Q is q_descale * decode(q) and
+ * likewise for K, and the scores are
+ *   s2[r,c] = fp32(decode(q_r) . decode(k_c)) * fp32(softmax_scale * q_descale * k_descale * log2 e)
+ * with every rule of ssa_fwd unchanged after that.
+ *   q, k        device E4M3 bytes [total_tokens, num_heads, 128] (head_dim must be 128)
+ *   v, out      device bf16 [total_tokens, num_heads, 128]
+ *   q_descale, k_descale  > 0, finite
+ *   skip_counter, decision_bitmap, tile_stat  as in ssa_fwd_ex, each nullable
+ * Returns SSA_OK or a negative status (SSA_ERR_UNSUPPORTED for head_dim != 128).
+ */
+int ssa_fwd_fp8(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch, int total_tokens,
+                int max_seqlen, int num_heads, int head_dim, float softmax_scale, float q_descale, float k_descale,
+                float threshold_scale_factor, void* out, int32_t* skip_counter, uint32_t* decision_bitmap,
+                float* tile_stat, void* stream);
+
+/*
+ * Per-tensor E4M3 quantisation for ssa_fwd_fp8: y[i] = E4M3(fp32(x[i] * inv_scale)),
+ * round to nearest even, saturating to +-448 (a caller with amax = max|x|
+ * passes inv_scale = 448 / amax and then q_descale = 1 / inv_scale).
+ *   x  device bf16 [n], 16-byte aligned;  y  device bytes [n], 8-byte aligned
+ * Returns SSA_OK, SSA_ERR_INVALID_ARG (n < 0, inv_scale not finite and > 0,
+ * NULL with n > 0) or SSA_ERR_UNSUPPORTED (misaligned pointer).
+ */
+int ssa_quantize_fp8(const void* x, void* y, int64_t n, float inv_scale, void* stream);
+
+/*
  * threshold_scale_factor = a * exp(b * target_sparsity) (README, "Calibrated
  * threshold"; TRT-LLM VisualGen docs, "Checkpoint Config"). Returns NaN when
  * a <= 0, target_sparsity is outside [0, 1] or an argument is not finite.

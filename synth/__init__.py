@@ -116,6 +116,54 @@ def f32_to_bf16(a: np.ndarray) -> np.ndarray:
     return ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
 
 
+# --- E4M3 (OCP 8-bit floating point, the variant without infinities) -------
+# 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits; exponent 0 holds the
+# subnormals m * 2^-9; S.1111.111 is NaN; the largest finite value is 448.
+# Used to prepare 8-bit Q/K inputs: every E4M3 value is exact in bf16.
+E4M3_MAX = 448.0
+
+
+def e4m3_to_f32(codes: np.ndarray) -> np.ndarray:
+    """Exact value of E4M3 codes (uint8) as float32 (NaN for the NaN codes)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int32)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    val = sign * mag
+    return np.where((e == 15) & (m == 7), np.nan, val).astype(np.float32)
+
+
+_E4M3_POS = e4m3_to_f32(np.arange(127, dtype=np.uint8)).astype(np.float64)  # codes 0..126, increasing
+
+
+def f32_to_e4m3(x: np.ndarray) -> np.ndarray:
+    """Round finite float32 values to E4M3 codes: nearest, ties to the even
+    code, magnitudes beyond 448 saturate to 448, the sign is kept (-0 -> 0x80)."""
+    x = np.asarray(x, dtype=np.float32)
+    a = np.abs(x.astype(np.float64))
+    hi = np.clip(np.searchsorted(_E4M3_POS, a, side="left"), 0, 126)  # first value >= a
+    lo = np.clip(hi - 1, 0, 126)
+    d_hi = _E4M3_POS[hi] - a
+    d_lo = a - _E4M3_POS[lo]
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(a >= _E4M3_POS[126], 126, code)
+    code = np.where(a <= 0.0, 0, code)
+    return (code | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)
+
+
+def quantize_e4m3(bf16_codes: np.ndarray):
+    """Per-tensor E4M3 quantisation of a bf16 tensor: inv_scale = fp32(448 / amax),
+    codes = E4M3(fp32(x * inv_scale)). Returns (codes, inv_scale as float32,
+    descale = 1 / inv_scale as float32)."""
+    x = bf16_to_f32(bf16_codes)
+    amax = float(np.max(np.abs(x)))
+    inv = np.float32(E4M3_MAX / amax)
+    codes = f32_to_e4m3(x * inv)  # float32 product, rounded once
+    return codes, inv, np.float32(1.0 / np.float64(inv))
+
+
 # Workloads: the tiny case the oracle finishes whole, the WAN-5B-like and the
 # WAN-14B 720p self-attention shapes, the calibration sweep and a varlen batch.
 TINY = Workload("tiny B1 H2 D64 S1024 grid 4x16x16", [(4, 16, 16)], H=2, D=64, seed=0, tsf=[0.0, 100.0, 1000.0])

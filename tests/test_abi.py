@@ -107,3 +107,29 @@ def test_resolve_and_fit_match_oracle(ssa):
     np.testing.assert_allclose(got, ref, rtol=1e-12)
     with pytest.raises(ssa.SSAError):
         ssa.fit_logspace([0.5, 0.5], [1.0, 1.0])
+
+
+def test_fp8_entry_points_validate_on_the_host(ssa):
+    L = ssa.lib()
+    fake = ctypes.c_void_p(0x10000)
+    mis = ctypes.c_void_p(0x10008)
+
+    def f8(D=128, qd=1.0, kd=1.0, total=256, q=fake, tsf=0.0):
+        return L.ssa_fwd_fp8(q, fake, fake, fake, 1, total, 256, 2, D, 0.0, qd, kd, tsf, fake, None, None, None, None)
+
+    assert f8(D=64) == ssa.SSA_ERR_UNSUPPORTED  # E4M3 rows must be 128 bytes
+    assert f8(qd=0.0) == ssa.SSA_ERR_INVALID_ARG
+    assert f8(kd=-1.0) == ssa.SSA_ERR_INVALID_ARG
+    assert f8(qd=float("inf")) == ssa.SSA_ERR_INVALID_ARG
+    assert f8(q=None) == ssa.SSA_ERR_INVALID_ARG
+    assert f8(q=mis) == ssa.SSA_ERR_UNSUPPORTED
+    assert f8(tsf=float("nan")) == ssa.SSA_ERR_INVALID_ARG
+    assert f8(total=0) == ssa.SSA_OK
+    qz = lambda x, y, n, s: L.ssa_quantize_fp8(x, y, n, s, None)
+    assert qz(fake, fake, -1, 1.0) == ssa.SSA_ERR_INVALID_ARG
+    assert qz(fake, fake, 16, 0.0) == ssa.SSA_ERR_INVALID_ARG
+    assert qz(fake, fake, 16, float("inf")) == ssa.SSA_ERR_INVALID_ARG
+    assert qz(None, fake, 16, 1.0) == ssa.SSA_ERR_INVALID_ARG
+    assert qz(mis, fake, 16, 1.0) == ssa.SSA_ERR_UNSUPPORTED
+    assert qz(fake, ctypes.c_void_p(0x10004), 16, 1.0) == ssa.SSA_ERR_UNSUPPORTED
+    assert qz(fake, fake, 0, 1.0) == ssa.SSA_OK

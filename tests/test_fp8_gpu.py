@@ -1,0 +1,110 @@
+"""GPU parity of the 8-bit Q/K forward (ssa_fwd_fp8) and of the E4M3
+quantiser (ssa_quantize_fp8). The oracle runs the same walk on the exactly
+decoded E4M3 values (each is exact in bf16) with the per-tensor descales
+folded into the softmax scale, which is how the scores are defined for this
+variant; outputs, decisions and skip counts are held to the same rules as
+the bf16 forward."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests import parity
+from tests.test_parity_gpu import Case, check_forward
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def ssa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import block_sparse_flashattention_ssa_b200 as m
+
+    assert m.get_error() == m.SSA_OK
+    return m
+
+
+def _device_codes(ssa, bf16_codes, inv):
+    x = torch.from_numpy(bf16_codes.view(np.int16)).to("cuda").view(torch.bfloat16)
+    return ssa.quantize_fp8(x, float(inv))
+
+
+class Fp8Case(Case):
+    """Q and K quantised per tensor on the GPU; the oracle sees their exact
+    decoded values and the descales inside the softmax scale."""
+
+    def __init__(self, ssa, w):
+        q, k, v = synth.generate(w)
+        self.q8, self.q_inv, self.q_ds = synth.quantize_e4m3(q)
+        self.k8, self.k_inv, self.k_ds = synth.quantize_e4m3(k)
+        dec = lambda c: synth.f32_to_bf16(synth.e4m3_to_f32(c))
+        super().__init__(ssa, w, dec(self.q8), dec(self.k8), v)
+        self.dq8 = _device_codes(ssa, q, self.q_inv)
+        self.dk8 = _device_codes(ssa, k, self.k_inv)
+        torch.cuda.synchronize()
+        assert np.array_equal(self.dq8.cpu().numpy(), self.q8) and np.array_equal(self.dk8.cpu().numpy(), self.k8)
+        # oracle softmax scale: 1/sqrt(D) * q_descale * k_descale, in the order the library forms it
+        self.scale = 1.0 / math.sqrt(w.D) * (float(self.q_ds) * float(self.k_ds))
+
+    def fwd(self, tsf, ex=True):
+        H = self.w.H
+        skip = torch.full((H, self.Q), -1, dtype=torch.int32, device="cuda")
+        bitmap = torch.zeros((H, self.Q, self.ssa.bitmap_words(self.w.max_seqlen)), dtype=torch.int32, device="cuda")
+        stat = torch.full((H, self.Q, self.T), float("nan"), dtype=torch.float32, device="cuda")
+        out = torch.full_like(self.dv, float("nan"))
+        self.ssa.fwd_fp8(self.dq8, self.dk8, self.dv, self.dcu, self.w.max_seqlen, float(self.q_ds),
+                         float(self.k_ds), tsf, out=out, skip_counter=skip, decision_bitmap=bitmap if ex else None,
+                         tile_stat=stat if ex else None)
+        self.ssa.check_device()
+        return (parity.bf16_host(out), skip.cpu().numpy(), bitmap.cpu().numpy().view(np.uint32),
+                stat.cpu().numpy())
+
+
+def _check(case, tsf, units=None, what=""):
+    out, skip, bitmap, stat = case.fwd(tsf)
+    res = oracle.walk(case.q, case.k, case.v, case.cu, case.w.H, case.w.D, softmax_scale=case.scale, tsf=tsf,
+                      units=units, max_tiles=case.T)
+    st = parity.Stats()
+    parity.compare_forward(res, case.cu, case.L_seq(tsf), out, skip, bitmap, stat, st, what=f"{what} tsf={tsf}")
+    st.check(f"{what} tsf={tsf}")
+    return st, skip
+
+
+def test_quantiser_matches_the_format_definition_bit_for_bit(ssa):
+    rng = np.random.default_rng(9)
+    n = 1_000_003  # not a multiple of 8: the scalar tail runs too
+    x = (rng.standard_normal(n) * np.exp2(rng.uniform(-14, 12, n))).astype(np.float32)
+    xb = synth.f32_to_bf16(x)
+    for inv in [1.0, 0.37, 61.5]:
+        got = _device_codes(ssa, xb, inv).cpu().numpy()
+        want = synth.f32_to_e4m3(synth.bf16_to_f32(xb) * np.float32(inv))
+        assert np.array_equal(got, want), inv
+
+
+def test_fp8_ragged_varlen(ssa):
+    lengths = [1, 5, 127, 128, 129, 300, 0, 1000]
+    w = synth.Workload("ragged fp8", [(1, 1, s) for s in lengths], H=3, D=128, seed=12, amp=3.0)
+    case = Fp8Case(ssa, w)
+    for tsf in [0.0, 50.0, 300.0, 2000.0]:
+        _check(case, tsf, what="ragged fp8")
+
+
+def test_fp8_wan5b_sampled(ssa):
+    case = Fp8Case(ssa, synth.WAN5B)
+    units = oracle.sample_units(case.cu, case.w.H, 24, seed=4)
+    for tsf in [0.0, 5e3, 2e4]:
+        _check(case, tsf, units=units, what="wan5b fp8")
+
+
+def test_fp8_skip_path_without_skips_is_bitwise_dense(ssa):
+    w = synth.Workload("fp8 bitwise", [(2, 16, 32)], H=2, D=128, seed=3, amp=3.0)
+    case = Fp8Case(ssa, w)
+    dense = case.fwd(0.0, ex=False)
+    tiny = case.fwd(1e-30, ex=False)
+    np.testing.assert_array_equal(dense[0], tiny[0])
+    assert tiny[1].sum() == 0
