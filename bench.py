@@ -251,11 +251,28 @@ def run_ours(args):
         r = float(skip.sum().item()) / tiles
         rows[name] = dict(tsf=t, ms=ms, skip_ratio=r, dense_eq_tflops=dense_flop / ms / 1e9,
                           effective_tflops=algorithmic_flop(w.seqlens, w.D, w.H, r) / ms / 1e9)
+    # side rows of the E4M3 Q/K variant (ssa_fwd_fp8) at the same thresholds
+    if fit is not None and w.D == 128:
+        _, q_inv, q_ds = synth.quantize_e4m3(q)
+        _, k_inv, k_ds = synth.quantize_e4m3(k)
+        dq8, dk8 = ssa.quantize_fp8(dq, float(q_inv)), ssa.quantize_fp8(dk, float(k_inv))
+        step8 = lambda t: ssa.fwd_fp8(dq8, dk8, dv, dcu, w.max_seqlen, float(q_ds), float(k_ds), t, out=out,
+                                      skip_counter=skip)
+        for name, t in [("fp8_qk_dense", 0.0), (f"fp8_qk_target_{HEADLINE_TARGET}", tsf)]:
+            for _ in range(2):
+                step8(t)
+            ms = statistics.median(time_fwd(ssa, lambda: step8(t), 5, stream))
+            ssa.check_device()
+            r = float(skip.sum().item()) / tiles
+            rows[name] = dict(tsf=t, ms=ms, skip_ratio=r, dense_eq_tflops=dense_flop / ms / 1e9,
+                              qk_dtype="e4m3 (per-tensor descale)")
+        del dq8, dk8
     dense_ms = rows["dense"]["ms"] if "dense" in rows else None
     for name, r in rows.items() if dense_ms else []:
-        r["speedup_vs_dense"] = dense_ms / r["ms"]
+        base = rows["fp8_qk_dense"]["ms"] if name.startswith("fp8") else dense_ms  # same-precision dense
+        r["speedup_vs_dense"] = base / r["ms"]
         if r["skip_ratio"] > 0:
-            r["f"] = (1.0 - r["ms"] / dense_ms) / r["skip_ratio"]
+            r["f"] = (1.0 - r["ms"] / base) / r["skip_ratio"]
 
     # timed region
     for _ in range(args.warmup):
