@@ -373,7 +373,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       int v_used = 0;
       for (int j = 0; ok && j < nkv; ++j) {
         const int t = j + 1;  // S_X(t) is issued right behind O_X += P_X(j) V_j
-        bool v_waited = false, k_waited = false;
+        // Waits that are normally already satisfied (K_{j+1}; in the dense and
+        // calibration orders also V_j) come first, while no MMA of this tile
+        // is in flight: a wait behind in-flight MMAs stalls the issuer.
+        if (t < nkv && !(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag))) break;
+        bool v_waited = false;
+        if (MODE != kSkip) {
+          if (!(ok = wait_bar(v_full(v_used % kVStages), (v_used / kVStages) & 1, abort_flag))) break;
+          v_waited = true;
+        }
         for (int x = 0; x < nx; ++x) {
           bool skip = false;
           if (MODE == kSkip) {
@@ -392,10 +400,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++kept[x];
           }
           if (t < nkv) {
-            if (!k_waited) {
-              if (!(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag))) break;
-              k_waited = true;
-            }
             tc_fence_after();
             issue_qk(x, t);
           }
