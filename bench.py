@@ -334,12 +334,9 @@ def run_ours(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) + 3-D sinusoidal positional code, amplitude 3)",
-        "config": {"workload": w.name, "global_batch": world, "seq_len": w.max_seqlen, "heads": w.H,
-                   "head_dim": w.D,
-                   "parallelism": f"dp{world} (independent problems, no collective)",
-                   "threshold": (f"tsf={tsf:.6g} resolved at target_sparsity {HEADLINE_TARGET} from a*exp(b*s) "
-                                 f"fitted by ssa_calibrate+ssa_fit_logspace on this input") if fit else f"tsf={tsf:g}",
-                   "l2": f"inputs larger than L2 ({3 * q.nbytes / 1e9:.2f} GB of Q/K/V per step)"},
+        "config": bench_config(w, world, (f"tsf={tsf:.6g} resolved at target_sparsity {HEADLINE_TARGET} from "
+                                          f"a*exp(b*s) fitted by ssa_calibrate+ssa_fit_logspace on this input")
+                               if fit else f"tsf={tsf:g}"),
         "skip_ratio": skip_ratio,
         "speedup_vs_dense": dense_ms / (total_ms / args.steps) if dense_ms else 1.0,
         "effective_tflops": achieved,
@@ -358,7 +355,7 @@ def run_ours(args):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(w, q, k, v, budget_s=args.cpu_seconds)
+        result["cpu_baseline"] = cpu_baseline(w, q, k, v, budget_s=args.cpu_seconds, tsf=tsf)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
@@ -367,6 +364,28 @@ def run_ours(args):
 
 
 # ------------------------------------------------------------ oracle (CPU)
+
+def bench_config(w, world, threshold):
+    """The `config` object of the JSON line (both arms)."""
+    return {"workload": w.name, "global_batch": world, "seq_len": w.max_seqlen, "heads": w.H, "head_dim": w.D,
+            "parallelism": f"dp{world} (independent problems, no collective)", "threshold": threshold,
+            "l2": f"inputs larger than L2 ({3 * w.total_tokens * w.H * w.D * 2 / 1e9:.2f} GB of Q/K/V per step)"}
+
+
+def oracle_threshold(w, q, k, v, target, n_units=16, seed=7):
+    """The oracle's own threshold for `target`: its calibration counts on a
+    sample of units, its log-space fit, its resolve (no GPU involved)."""
+    import oracle
+    import synth
+
+    units = oracle.sample_units(w.cu_seqlens, w.H, n_units, seed=seed)
+    res = oracle.walk(q, k, v, w.cu_seqlens, w.H, w.D, units=units, cal_lambdas=synth.CALIB_THRESHOLDS,
+                      nthreads=os.cpu_count() or 1)
+    nkv = (w.seqlens[0] + TILE - 1) // TILE
+    sparsity = res["counts"].sum(axis=0) / (len(units) * nkv)
+    a, b, _, _ = oracle.fit_logspace(sparsity, [lam * w.seqlens[0] for lam in synth.CALIB_THRESHOLDS])
+    return oracle.resolve(a, b, target)
+
 
 def cpu_baseline(w, q, k, v, budget_s=12.0, tsf=None):
     """The CPU oracle as it stands, on a bounded sample of (head, q-block)
@@ -391,7 +410,7 @@ def cpu_baseline(w, q, k, v, budget_s=12.0, tsf=None):
     flop = 4.0 * rows * S * w.D
     return {"value": flop / dt / 1e12, "unit": "TFLOP/s (dense-equivalent)", "cores": cores, "kind": "oracle",
             "sample": f"{done} (head, q-block) units of the S=75,600 workload ({rows} query rows, "
-                      f"{dt:.1f} s wall), dense threshold"}
+                      f"{dt:.1f} s wall), tsf={tsf or 0.0:.6g}"}
 
 
 def run_reference(args):
@@ -405,10 +424,11 @@ def run_reference(args):
     q, k, v = synth.generate(w)
     for _ in range(args.warmup):
         pass  # the oracle has no warm-up state; warm-up steps are free
+    tsf = oracle_threshold(w, q, k, v, HEADLINE_TARGET)  # not timed
     per = []
     cb = None
     for _ in range(args.steps):
-        cb = cpu_baseline(w, q, k, v, budget_s=args.cpu_seconds / max(args.steps, 1))
+        cb = cpu_baseline(w, q, k, v, budget_s=args.cpu_seconds / max(args.steps, 1), tsf=tsf)
         per.append(cb["value"])
     value = statistics.mean(per)
     full_ms = w.dense_flop() / (value * 1e12) * 1e3
@@ -418,8 +438,9 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": full_ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) + 3-D sinusoidal positional code, amplitude 3)",
-        "config": {"workload": "WAN-14B 720p self-attention B1 H40 D128 S75600 (grid 21x45x80)",
-                   "note": "each step is a bounded sample of the workload; ms_per_step is extrapolated"},
+        "config": dict(bench_config(w, world, f"tsf={tsf:.6g} resolved at target_sparsity {HEADLINE_TARGET} from "
+                                              f"the oracle's own calibration and fit on 16 sampled units"),
+                       note="each step is a bounded sample of the workload; ms_per_step is extrapolated"),
         "cpu_baseline": cb,
         "e2e": {"value": value, "unit": "TFLOP/s (dense-equivalent)", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
