@@ -16,7 +16,8 @@
 //           to keep tile j (a tile both skip issues no V load);
 //   warp 9  tcgen05 issuer, per KV tile j and per block X in order A, B:
 //           O_X += P_X V_j (when X keeps j, P_X read from TMEM), then
-//           S_X = Q_X K_{j+1}^T into the same TMEM columns.
+//           S_X = Q_X K_{j+1}^T into the same TMEM columns (bf16 operands, or
+//           E4M3 ones with per-tensor descales folded into the score scale).
 // tcgen05 MMAs issued by one thread execute in issue order, so the S MMA
 // cannot overwrite P_X before the PV MMA ahead of it has read P_X; and a
 // commit tracks every earlier MMA of the thread, so when S_X(j+1) is reported
