@@ -114,6 +114,51 @@ def _shape(q):
     return q.shape[0], q.shape[1], q.shape[2]
 
 
+def _require(t, name, dtype, device, shape=None, allow_none=False):
+    """Host-side check of a tensor argument: on the device of q, contiguous,
+    of the expected dtype (and shape). A host tensor handed to the kernels
+    would fault the GPU, so this is checked before the library is called."""
+    import torch
+
+    if t is None:
+        if allow_none:
+            return
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _check_attention_args(q, k, v, cu_seqlens, out, qk_dtype):
+    import torch
+
+    if not (isinstance(q, torch.Tensor) and q.is_cuda):
+        raise ValueError("q must be a CUDA tensor")
+    dev = q.device
+    shape = tuple(q.shape)
+    _require(q, "q", qk_dtype, dev)
+    _require(k, "k", qk_dtype, dev, shape)
+    _require(v, "v", torch.bfloat16, dev, shape)
+    _require(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens must be a 1-D tensor of batch + 1 offsets")
+    _require(out, "out", torch.bfloat16, dev, shape, allow_none=True)
+    return dev
+
+
+def _check_per_unit(t, name, dtype, dev, H):
+    _require(t, name, dtype, dev, allow_none=True)
+    if t is not None and (t.dim() < 2 or t.shape[0] != H):
+        raise ValueError(f"{name} must be [num_heads, num_qblocks, ...] with num_heads = {H}")
+
+
 def num_qblocks(cu_seqlens) -> int:
     """Total 128-row query blocks over the batch (from a host copy of cu_seqlens)."""
     cu = np.ascontiguousarray(np.asarray(cu_seqlens if not hasattr(cu_seqlens, "cpu") else cu_seqlens.cpu()),
@@ -135,6 +180,10 @@ def fwd(q, k, v, cu_seqlens, max_seqlen: int, threshold_scale_factor: float = 0.
     import torch
 
     total, H, D = _shape(q)
+    dev = _check_attention_args(q, k, v, cu_seqlens, out, torch.bfloat16)
+    _check_per_unit(skip_counter, "skip_counter", torch.int32, dev, H)
+    _check_per_unit(decision_bitmap, "decision_bitmap", (torch.int32, torch.uint32), dev, H)
+    _check_per_unit(tile_stat, "tile_stat", torch.float32, dev, H)
     if out is None:
         out = torch.empty_like(q)
     batch = cu_seqlens.numel() - 1
@@ -156,6 +205,10 @@ def fwd_fp8(q8, k8, v, cu_seqlens, max_seqlen: int, q_descale: float, k_descale:
     import torch
 
     total, H, D = _shape(q8)
+    dev = _check_attention_args(q8, k8, v, cu_seqlens, out, torch.uint8)
+    _check_per_unit(skip_counter, "skip_counter", torch.int32, dev, H)
+    _check_per_unit(decision_bitmap, "decision_bitmap", (torch.int32, torch.uint32), dev, H)
+    _check_per_unit(tile_stat, "tile_stat", torch.float32, dev, H)
     if out is None:
         out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
     batch = cu_seqlens.numel() - 1
@@ -171,6 +224,10 @@ def quantize_fp8(x, inv_scale: float, out=None, stream=None):
     """E4M3 codes (uint8, same shape) of fp32(x * inv_scale), nearest even, saturating."""
     import torch
 
+    if not (isinstance(x, torch.Tensor) and x.is_cuda):
+        raise ValueError("x must be a CUDA tensor")
+    _require(x, "x", torch.bfloat16, x.device)
+    _require(out, "out", torch.uint8, x.device, tuple(x.shape), allow_none=True)
     if out is None:
         out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     _check(_lib.ssa_quantize_fp8(_ptr(x), _ptr(out), x.numel(), float(inv_scale), _stream_handle(stream)),
@@ -186,7 +243,11 @@ def calibrate(q, k, v, cu_seqlens, max_seqlen: int, thresholds, softmax_scale: f
     import torch
 
     total, H, D = _shape(q)
+    dev = _check_attention_args(q, k, v, cu_seqlens, out, torch.bfloat16)
+    _check_per_unit(counts, "counts", torch.int32, dev, H)
     th = np.ascontiguousarray(thresholds, dtype=np.float32)
+    if counts is not None and (counts.dim() != 3 or counts.shape[2] != len(th)):
+        raise ValueError("counts must be [num_heads, num_qblocks, n_thresholds]")
     if out is None:
         out = torch.empty_like(q)
     if counts is None:

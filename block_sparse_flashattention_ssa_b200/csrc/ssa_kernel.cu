@@ -40,6 +40,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <initializer_list>
 
 #include "sm100.cuh"
 #include "ssa.h"
@@ -659,6 +660,28 @@ struct Call {
   double qk_descale = 1.0;      // q_descale * k_descale (E4M3 only)
 };
 
+// True when `p` is device (or managed) memory of the current device: a host
+// pointer handed to a kernel or a tensor map would fault the GPU, so every
+// pointer the kernels touch is checked before a launch.
+bool on_current_device(const void* ptr) {
+  if (!ptr) return false;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  cudaPointerAttributes attr{};
+  if (cudaPointerGetAttributes(&attr, ptr) != cudaSuccess) {
+    cudaGetLastError();  // clear the error this query may leave behind
+    return false;
+  }
+  return (attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged) && attr.device == dev;
+}
+
+// Every non-null pointer of `ptrs` lives on the current device.
+int check_device_pointers(std::initializer_list<const void*> ptrs) {
+  for (const void* ptr : ptrs)
+    if (ptr && !on_current_device(ptr)) return SSA_ERR_INVALID_ARG;
+  return SSA_OK;
+}
+
 // Host-side argument check. total_tokens == 0 is a valid no-op whatever the
 // data pointers are (an empty batch has no storage).
 int validate(const Call& a) {
@@ -672,7 +695,7 @@ int validate(const Call& a) {
   if (!a.q || !a.k || !a.v || !a.out) return SSA_ERR_INVALID_ARG;
   for (const void* ptr : {a.q, a.k, a.v, static_cast<const void*>(a.out)})
     if (reinterpret_cast<uintptr_t>(ptr) & 15u) return SSA_ERR_UNSUPPORTED;
-  return SSA_OK;
+  return check_device_pointers({a.q, a.k, a.v, a.out, a.cu});
 }
 
 Params base_params(const Call& a) {
@@ -753,6 +776,7 @@ int fwd_impl(const Call& a, float tsf, int32_t* skip_counter, uint32_t* bitmap, 
   if (std::isnan(tsf) || std::isinf(tsf)) return SSA_ERR_INVALID_ARG;
   if ((bitmap || tile_stat) && a.max_seqlen < 1) return SSA_ERR_INVALID_ARG;
   if (a.total_tokens == 0) return SSA_OK;
+  if ((rc = check_device_pointers({skip_counter, bitmap, tile_stat})) != SSA_OK) return rc;
   Params p = base_params(a);
   p.skip_counter = skip_counter;
   p.bitmap = bitmap;
@@ -786,6 +810,7 @@ extern "C" int ssa_quantize_fp8(const void* x, void* y, int64_t n, float inv_sca
   if (n == 0) return SSA_OK;
   if (!x || !y) return SSA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(y) & 7u)) return SSA_ERR_UNSUPPORTED;
+  if (const int rc = check_device_pointers({x, y}); rc != SSA_OK) return rc;
   const int64_t groups = n / 8;
   const int threads = 256;
   const int64_t want = (groups + threads - 1) / threads;
@@ -824,6 +849,7 @@ extern "C" int ssa_calibrate(const void* q, const void* k, const void* v, const 
   for (int i = 0; i < n_thresholds; ++i)
     if (!(thresholds[i] > 0.f) || std::isinf(thresholds[i])) return SSA_ERR_INVALID_ARG;
   if (total_tokens == 0) return SSA_OK;
+  if ((rc = check_device_pointers({counts})) != SSA_OK) return rc;
   Params p = base_params(a);
   p.counts = counts;
   p.n_cal = n_thresholds;
@@ -835,6 +861,7 @@ extern "C" const char* ssa_last_cuda_error(void) { return t_last_cuda_error; }
 
 extern "C" int ssa_wait_timeout_check(int* result, int64_t limit_ns, void* stream) {
   if (!result || limit_ns <= 0 || limit_ns > 1000000000) return SSA_ERR_INVALID_ARG;
+  if (const int rc = check_device_pointers({result}); rc != SSA_OK) return rc;
   wait_timeout_check_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(limit_ns), result);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? SSA_OK : cuda_fail(e);

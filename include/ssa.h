@@ -37,7 +37,11 @@
  * synchronising. Errors a kernel detects (an inconsistent cu_seqlens, a
  * device wait that ran past its time limit) are recorded in a per-device
  * status word that ssa_get_error() reads. Q, K, V and out must be 16-byte
- * aligned.
+ * aligned. Every pointer documented as a device pointer must be device (or
+ * managed) memory of the current device: the entry points check this with
+ * cudaPointerGetAttributes before any launch and return SSA_ERR_INVALID_ARG
+ * otherwise. Buffer sizes cannot be checked: the caller sizes the per-unit
+ * outputs from ssa_num_qblocks().
  */
 #ifndef SSA_H_
 #define SSA_H_

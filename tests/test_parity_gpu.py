@@ -185,3 +185,37 @@ def test_empty_inputs_and_device_side_argument_check(ssa):
     assert ssa.get_error() == ssa.SSA_ERR_DEVICE_ARG
     assert bool((out == 7.0).all())
     assert ssa.get_error() == ssa.SSA_OK  # the status word was cleared
+
+
+def test_host_memory_is_refused_before_any_launch(ssa):
+    """Arguments that are not device memory of the current device never
+    reach a kernel: the binding rejects host tensors, and the C entry points
+    reject host pointers (checked here with pinned, device-mapped host
+    memory, which a kernel could read without faulting, so the test cannot
+    fault the GPU even if the check were missing)."""
+    import ctypes
+
+    w = synth.Workload("one", [(1, 1, 200)], H=2, D=64, seed=0)
+    case = Case(ssa, w)
+    with pytest.raises(ValueError):
+        ssa.fwd(case.dq.cpu(), case.dk, case.dv, case.dcu, 200, 10.0)
+    with pytest.raises(ValueError):
+        ssa.fwd(case.dq, case.dk, case.dv, case.dcu.cpu(), 200, 10.0)
+    with pytest.raises(ValueError):
+        ssa.fwd(case.dq, case.dk, case.dv, case.dcu, 200, 10.0,
+                skip_counter=torch.zeros((2, 2), dtype=torch.int32).pin_memory())
+    L = ssa.lib()
+    vp = ctypes.c_void_p
+    out = torch.full_like(case.dq, 7.0)
+    host_cu = torch.tensor([0, 200], dtype=torch.int32).pin_memory()
+    host_skip = torch.full((2, 2), -1, dtype=torch.int32).pin_memory()
+    stream = vp(torch.cuda.current_stream().cuda_stream)
+    rc = L.ssa_fwd(vp(case.dq.data_ptr()), vp(case.dk.data_ptr()), vp(case.dv.data_ptr()), vp(host_cu.data_ptr()),
+                   1, 200, 200, 2, 64, 0.0, 10.0, vp(out.data_ptr()), None, stream)
+    assert rc == ssa.SSA_ERR_INVALID_ARG
+    rc = L.ssa_fwd(vp(case.dq.data_ptr()), vp(case.dk.data_ptr()), vp(case.dv.data_ptr()), vp(case.dcu.data_ptr()),
+                   1, 200, 200, 2, 64, 0.0, 10.0, vp(out.data_ptr()), vp(host_skip.data_ptr()), stream)
+    assert rc == ssa.SSA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert ssa.get_error() == ssa.SSA_OK
+    assert bool((out == 7.0).all()) and bool((host_skip == -1).all())  # nothing ran
