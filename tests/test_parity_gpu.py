@@ -166,6 +166,24 @@ def test_calibration_wan5b_sampled(ssa):
     check_calibration(case, units=units, what="calib wan5b")
 
 
+def test_calibration_varlen_sampled(ssa):
+    """Calibration counts over a packed batch of sequences of different
+    lengths (each unit counts against its own sequence's tiles)."""
+    case = Case(ssa, synth.VARLEN)
+    units = oracle.sample_units(case.cu, case.w.H, 16, seed=5)
+    check_calibration(case, units=units, what="calib varlen")
+
+
+def test_d64_long_sequence_sampled(ssa):
+    """D = 64 at S = 8192 (the WAN-5B-like grid, 16 heads): dense and two
+    thresholds (lambda below and above 1), 24 sampled units each."""
+    w = synth.Workload("D64 S8192", [(8, 32, 32)], H=16, D=64, seed=11, amp=3.0)
+    case = Case(ssa, w)
+    units = oracle.sample_units(case.cu, w.H, 24, seed=6)
+    for tsf in [0.0, 3000.0, 12000.0]:
+        check_forward(case, tsf, units=units, what="d64 s8192")
+
+
 def test_empty_inputs_and_device_side_argument_check(ssa):
     w = synth.Workload("one", [(1, 1, 200)], H=2, D=64, seed=0)
     case = Case(ssa, w)
