@@ -151,7 +151,7 @@ def init_dist(world, backend):
 
     if world > 1 and not dist.is_initialized():
         os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
-        dist.init_process_group(backend, timeout=timedelta(seconds=300))
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
     return dist
 
 
