@@ -58,6 +58,7 @@ constexpr int kMmaWarp = 9;
 constexpr int kThreads = 320;
 constexpr int kKStages = 3;
 constexpr int kVStages = 2;
+constexpr int kCalWindow = 16;  // calibration: tiles whose votes are counted together
 constexpr int kDecRing = 4;  // > kKStages - 1: bounds how far a vote runs ahead of its readers
 constexpr uint32_t kTmemCols = 512;
 __host__ __device__ constexpr uint32_t col_S(int x) { return x ? 128u : 0u; }    // S_X (and P_X)
@@ -104,7 +105,7 @@ struct Ctl {
   int abort_flag;
   int dec[kQBlocks][kDecRing];
   float red[kQBlocks][2][4];
-  int cnt[kQBlocks][SSA_MAX_THRESHOLDS];  // calibration counts of each block (its group's first thread)
+  float cal_red[kQBlocks][2][kCalWindow][4];  // calibration: each warp's vote per tile, double-buffered windows
   int seq, qb_a, has_b, S, start, gqb_a, nq_total;
 };
 
@@ -124,6 +125,7 @@ struct Layout {
   static constexpr int kCtl = kV + kVStages * kVTileBytes;
   static constexpr int kBytes = kCtl + static_cast<int>(sizeof(Ctl));
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 B (128B swizzle atoms)
+  static_assert(kAlloc <= 232448, "shared memory beyond the 227 KB a CTA may use");
 };
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag,
@@ -439,8 +441,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_used = -INFINITY;  // reference max of the exponentials (lags m_true by < kRescaleThreshold)
     float l = 0.f;
     int kept = 0, nskip = 0;
-    if (MODE == kCalib && gt == 0)
-      for (int k = 0; k < SSA_MAX_THRESHOLDS; ++k) ctl.cnt[x][k] = 0;
+    // Calibration: thread gt counts tile slot (gt & 15) of every window for
+    // thresholds (gt >> 4) + 8m, m = 0..3 (up to 32 thresholds).
+    int cal_cnt[4] = {0, 0, 0, 0};
     uint32_t bits = 0;
     bool ok = true;
 
@@ -472,7 +475,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7])) * c;
 
       bool skip = false;
-      if (MODE != kDense || EX) {
+      if (MODE == kCalib) {
+        // No per-tile barrier: each warp leaves its vote in the current
+        // window; once per window (and after the last tile) the group meets
+        // and counts every threshold for the window's tiles in parallel.
+        const float dr = warp_max_f32(row_valid ? (tmax - m_true) : -INFINITY);
+        const int win = j / kCalWindow, slot = j % kCalWindow;
+        if (lane == 0) ctl.cal_red[x][win & 1][slot][wq] = dr;
+        if (slot == kCalWindow - 1 || j == nkv - 1) {
+          named_barrier_sync(vote_bar, 128);
+          const int i = gt & (kCalWindow - 1);
+          if (i <= slot) {
+            volatile float* r = ctl.cal_red[x][win & 1][i];
+            const float d = fmaxf(fmaxf(r[0], r[1]), fmaxf(r[2], r[3]));
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              const int k = (gt >> 4) + 8 * m;
+              if (k < p.n_cal) cal_cnt[m] += d < p.Lcal[k] ? 1 : 0;
+            }
+          }
+        }
+      } else if (MODE != kDense || EX) {
         const float dr = warp_max_f32(row_valid ? (tmax - m_true) : -INFINITY);
         if (lane == 0) ctl.red[x][j & 1][wq] = dr;
         // S_X(j) has been read into registers by every warp of the group once
@@ -482,9 +505,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         volatile float* red = ctl.red[x][j & 1];
         const float d = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
         if (MODE == kSkip) skip = d < Lthr;
-        if (MODE == kCalib && gt == 0) {
-          for (int k = 0; k < p.n_cal; ++k) ctl.cnt[x][k] += d < p.Lcal[k] ? 1 : 0;
-        }
         if (EX && gt == 0) {
           if (p.tile_stat) p.tile_stat[unit * p.max_tiles + j] = d;
           bits |= (skip ? 1u : 0u) << (j & 31);
@@ -583,12 +603,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (gt == 0) {
-        if (p.skip_counter) p.skip_counter[unit] = nskip;
-        if (MODE == kCalib) {
-          for (int k = 0; k < p.n_cal; ++k) p.counts[unit * p.n_cal + k] = ctl.cnt[x][k];
+      if (MODE == kCalib) {  // add over the 16 lanes that share thresholds; lanes 0 and 16 store
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          int v = cal_cnt[m];
+#pragma unroll
+          for (int o = 1; o < 16; o <<= 1) v += __shfl_xor_sync(kFull, v, o);
+          const int k = (gt >> 4) + 8 * m;
+          if ((lane & 15) == 0 && k < p.n_cal) p.counts[unit * p.n_cal + k] = v;
         }
       }
+      if (gt == 0 && p.skip_counter) p.skip_counter[unit] = nskip;
     }
   }
 
