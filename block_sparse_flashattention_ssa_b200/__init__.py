@@ -12,6 +12,7 @@ Entry points (same names as the C ABI, without the ``ssa_`` prefix):
   fwd_fp8      the forward with E4M3 Q and K (per-tensor descales)
   quantize_fp8 bf16 -> E4M3 per-tensor quantisation for fwd_fp8
   calibrate    dense attention + skip counts at N thresholds at once
+  calibrate_fp8  the same with E4M3 Q and K
   resolve      threshold_scale_factor = a * exp(b * target_sparsity)
   fit_logspace log-space least-squares fit of (a, b)
   num_qblocks  number of 128-row query blocks of a batch
@@ -58,6 +59,8 @@ def _load():
     L.ssa_fwd_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp, vp, vp]
     L.ssa_fwd_fp8.restype = i32
     L.ssa_fwd_fp8.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32, f32, vp, vp, vp, vp, vp]
+    L.ssa_calibrate_fp8.restype = i32
+    L.ssa_calibrate_fp8.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32, vp, i32, vp, vp, vp]
     L.ssa_quantize_fp8.restype = i32
     L.ssa_quantize_fp8.argtypes = [vp, vp, ctypes.c_int64, f32, vp]
     L.ssa_calibrate.restype = i32
@@ -258,6 +261,29 @@ def calibrate(q, k, v, cu_seqlens, max_seqlen: int, thresholds, softmax_scale: f
                             float(softmax_scale), th.ctypes.data, len(th), _ptr(out), _ptr(counts),
                             _stream_handle(stream))
     _check(rc, "ssa_calibrate")
+    return out, counts
+
+
+def calibrate_fp8(q8, k8, v, cu_seqlens, max_seqlen: int, q_descale: float, k_descale: float, thresholds,
+                  softmax_scale: float = 0.0, out=None, counts=None, stream=None):
+    """calibrate() on the E4M3 scores of fwd_fp8. Returns (out, counts[H, Q, N])."""
+    import torch
+
+    total, H, D = _shape(q8)
+    dev = _check_attention_args(q8, k8, v, cu_seqlens, out, torch.uint8)
+    _check_per_unit(counts, "counts", torch.int32, dev, H)
+    th = np.ascontiguousarray(thresholds, dtype=np.float32)
+    if counts is not None and (counts.dim() != 3 or counts.shape[2] != len(th)):
+        raise ValueError("counts must be [num_heads, num_qblocks, n_thresholds]")
+    if out is None:
+        out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    if counts is None:
+        counts = torch.empty((H, num_qblocks(cu_seqlens), len(th)), dtype=torch.int32, device=dev)
+    batch = cu_seqlens.numel() - 1
+    rc = _lib.ssa_calibrate_fp8(_ptr(q8), _ptr(k8), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D,
+                                float(softmax_scale), float(q_descale), float(k_descale), th.ctypes.data, len(th),
+                                _ptr(out), _ptr(counts), _stream_handle(stream))
+    _check(rc, "ssa_calibrate_fp8")
     return out, counts
 
 

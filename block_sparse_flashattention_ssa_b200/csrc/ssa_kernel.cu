@@ -863,23 +863,44 @@ extern "C" int ssa_fwd_ex(const void* q, const void* k, const void* v, const int
   return fwd_impl(a, threshold_scale_factor, skip_counter, decision_bitmap, tile_stat);
 }
 
-extern "C" int ssa_calibrate(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
-                             int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
-                             const float* thresholds, int n_thresholds, void* out, int32_t* counts, void* stream) {
-  const Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
-               static_cast<cudaStream_t>(stream)};
+namespace ssa {
+namespace {
+int calibrate_impl(const Call& a, const float* thresholds, int n_thresholds, int32_t* counts) {
   int rc = validate(a);
   if (rc != SSA_OK) return rc;
   if (!thresholds || !counts || n_thresholds < 1 || n_thresholds > SSA_MAX_THRESHOLDS) return SSA_ERR_INVALID_ARG;
   for (int i = 0; i < n_thresholds; ++i)
     if (!(thresholds[i] > 0.f) || std::isinf(thresholds[i])) return SSA_ERR_INVALID_ARG;
-  if (total_tokens == 0) return SSA_OK;
+  if (a.total_tokens == 0) return SSA_OK;
   if ((rc = check_device_pointers({counts})) != SSA_OK) return rc;
   Params p = base_params(a);
   p.counts = counts;
   p.n_cal = n_thresholds;
   for (int i = 0; i < n_thresholds; ++i) p.Lcal[i] = static_cast<float>(std::log2(static_cast<double>(thresholds[i])));
   return dispatch_d<kCalib, false>(a, p);
+}
+}  // namespace
+}  // namespace ssa
+
+extern "C" int ssa_calibrate(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                             int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                             const float* thresholds, int n_thresholds, void* out, int32_t* counts, void* stream) {
+  const Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
+               static_cast<cudaStream_t>(stream)};
+  return calibrate_impl(a, thresholds, n_thresholds, counts);
+}
+
+extern "C" int ssa_calibrate_fp8(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                                 int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                                 float q_descale, float k_descale, const float* thresholds, int n_thresholds,
+                                 void* out, int32_t* counts, void* stream) {
+  Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
+         static_cast<cudaStream_t>(stream)};
+  if (!(q_descale > 0.f) || !(k_descale > 0.f) || std::isinf(q_descale) || std::isinf(k_descale))
+    return SSA_ERR_INVALID_ARG;
+  a.f8 = true;
+  a.qk_descale = static_cast<double>(q_descale) * static_cast<double>(k_descale);
+  return calibrate_impl(a, thresholds, n_thresholds, counts);
 }
 
 extern "C" const char* ssa_last_cuda_error(void) { return t_last_cuda_error; }

@@ -145,6 +145,18 @@ int ssa_fwd_fp8(const void* q, const void* k, const void* v, const int32_t* cu_s
 int ssa_quantize_fp8(const void* x, void* y, int64_t n, float inv_scale, void* stream);
 
 /*
+ * ssa_calibrate with 8-bit Q and K: the dense pass and its counts on the
+ * scores ssa_fwd_fp8 defines (E4M3 Q, K with per-tensor descales; V and out
+ * bf16; head_dim 128). For lambda_k <= 1 the count equals ssa_fwd_fp8's skip
+ * count at threshold_scale_factor = lambda_k * S_kv. Arguments as in
+ * ssa_calibrate and ssa_fwd_fp8.
+ */
+int ssa_calibrate_fp8(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                      int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                      float q_descale, float k_descale, const float* thresholds, int n_thresholds, void* out,
+                      int32_t* counts, void* stream);
+
+/*
  * threshold_scale_factor = a * exp(b * target_sparsity) (README, "Calibrated
  * threshold"; TRT-LLM VisualGen docs, "Checkpoint Config"). Returns NaN when
  * a <= 0, target_sparsity is outside [0, 1] or an argument is not finite.

@@ -108,3 +108,33 @@ def test_fp8_skip_path_without_skips_is_bitwise_dense(ssa):
     tiny = case.fwd(1e-30, ex=False)
     np.testing.assert_array_equal(dense[0], tiny[0])
     assert tiny[1].sum() == 0
+
+
+def test_fp8_calibration_counts_and_forward_equivalence(ssa):
+    """ssa_calibrate_fp8 against the oracle's calibration walk on the decoded
+    values; its output is the dense E4M3 output; for lambda <= 1 its counts
+    equal ssa_fwd_fp8's skip counts at tsf = lambda * S (S = 1024, so the
+    threshold is the same float on both paths)."""
+    lams = synth.CALIB_THRESHOLDS
+    w = synth.Workload("calib fp8", [(1, 1, 300), (1, 1, 129), (1, 1, 1000)], H=2, D=128, seed=13, amp=3.0)
+    case = Fp8Case(ssa, w)
+    out, counts = ssa.calibrate_fp8(case.dq8, case.dk8, case.dv, case.dcu, w.max_seqlen, float(case.q_ds),
+                                    float(case.k_ds), lams)
+    ssa.check_device()
+    res = oracle.walk(case.q, case.k, case.v, case.cu, w.H, w.D, softmax_scale=case.scale, cal_lambdas=lams,
+                      max_tiles=case.T)
+    st = parity.Stats()
+    parity.compare_calibration(res, case.cu, [oracle.lambda_log2(x) for x in lams], parity.bf16_host(out),
+                               counts.cpu().numpy(), st, what="calib fp8")
+    st.check("calib fp8")
+    np.testing.assert_array_equal(parity.bf16_host(out), case.fwd(0.0, ex=False)[0])
+
+    w1 = synth.Workload("calib fp8 S1024", [(4, 16, 16)], H=2, D=128, seed=14, amp=3.0)
+    one = Fp8Case(ssa, w1)
+    _, c1 = ssa.calibrate_fp8(one.dq8, one.dk8, one.dv, one.dcu, w1.max_seqlen, float(one.q_ds), float(one.k_ds),
+                              lams)
+    ssa.check_device()
+    c1 = c1.cpu().numpy()
+    for kk, lam in enumerate(lams):
+        _, skip, _, _ = one.fwd(lam * 1024)
+        assert np.array_equal(skip, c1[:, :, kk]), lam
