@@ -29,6 +29,7 @@ from typing import Callable, List, Optional, Sequence
 import numpy as np
 
 from . import calibrate as _calibrate
+from . import calibrate_fp8 as _calibrate_fp8
 from . import fit_logspace as _fit_logspace
 from . import resolve as _resolve
 
@@ -114,12 +115,19 @@ def torch_allreduce(group=None) -> Callable[[np.ndarray], np.ndarray]:
 
 def calibrate(q, k, v, cu_seqlens, max_seqlen: int, trials: Sequence[float] = DEFAULT_TRIALS,
               softmax_scale: float = 0.0, total_heads: Optional[int] = None,
-              allreduce: Optional[Callable[[np.ndarray], np.ndarray]] = None, stream=None) -> Calibration:
+              allreduce: Optional[Callable[[np.ndarray], np.ndarray]] = None, descales=None,
+              stream=None) -> Calibration:
     """Count on the GPU, sum per sequence, optionally add the other ranks'
     sums (heads sharded: q, k, v hold this rank's heads, total_heads counts
-    all ranks'), and fit. Every rank that takes part gets the same result."""
-    _, counts = _calibrate(q, k, v, cu_seqlens, max_seqlen, list(trials), softmax_scale=softmax_scale,
-                           stream=stream)
+    all ranks'), and fit. Every rank that takes part gets the same result.
+    With ``descales = (q_descale, k_descale)``, q and k are E4M3 codes and the
+    counts come from ssa_calibrate_fp8."""
+    if descales is None:
+        _, counts = _calibrate(q, k, v, cu_seqlens, max_seqlen, list(trials), softmax_scale=softmax_scale,
+                               stream=stream)
+    else:
+        _, counts = _calibrate_fp8(q, k, v, cu_seqlens, max_seqlen, float(descales[0]), float(descales[1]),
+                                   list(trials), softmax_scale=softmax_scale, stream=stream)
     cu_host = cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else np.asarray(cu_seqlens)
     seq = sequence_counts(counts.cpu().numpy(), cu_host)
     if allreduce is not None:
