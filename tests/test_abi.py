@@ -23,9 +23,9 @@ def declared_entry_points():
 
 @pytest.fixture(scope="module")
 def ssa():
-    from block_sparse_flashattention_ssa_b200 import build
+    import __graft_entry__
 
-    build.build()
+    __graft_entry__._library_builder().build()
     import block_sparse_flashattention_ssa_b200 as m
 
     return m
