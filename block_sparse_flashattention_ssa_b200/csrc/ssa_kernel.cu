@@ -547,13 +547,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       uint32_t lo[64];
       tmem_ld_x64_async(lane_base + col_s, lo);  // lands while the upper half is exponentiated
-      uint32_t pk_hi[32];  // P columns [64,128) -> packed TMEM columns [32,64)
+      // Packed P: [0,32) from S columns [0,64), [32,64) from [64,128). The
+      // dense and calibration kernels store it with one 64-column store; the
+      // skipping kernel, which has less register room, with two.
+      uint32_t pk[64];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float2 a = ffma2(make_float2(__uint_as_float(hi[2 * i]), __uint_as_float(hi[2 * i + 1])), c2, nm2);
         const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
         rs[i & 1] = fadd2(rs[i & 1], e);
-        pk_hi[i] = pack_bf16x2(e.x, e.y);
+        pk[32 + i] = pack_bf16x2(e.x, e.y);
       }
       tmem_wait_ld_tied(lo);
       if (valid < 64) {
@@ -561,17 +564,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 64; ++i)
           if (i >= valid) lo[i] = __float_as_uint(-INFINITY);
       }
-      uint32_t pk_lo[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float2 a = ffma2(make_float2(__uint_as_float(lo[2 * i]), __uint_as_float(lo[2 * i + 1])), c2, nm2);
         const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
         rs[i & 1] = fadd2(rs[i & 1], e);
-        pk_lo[i] = pack_bf16x2(e.x, e.y);
+        pk[i] = pack_bf16x2(e.x, e.y);
       }
       // Both halves of S_X are in registers by now: P_X may overwrite them.
-      tmem_st_x32(lane_base + col_s, pk_lo);
-      tmem_st_x32(lane_base + col_s + 32, pk_hi);
+      if (MODE == kSkip) {
+        tmem_st_x32(lane_base + col_s, reinterpret_cast<const uint32_t(&)[32]>(pk[0]));
+        tmem_st_x32(lane_base + col_s + 32, reinterpret_cast<const uint32_t(&)[32]>(pk[32]));
+      } else {
+        tmem_st_x64(lane_base + col_s, pk);
+      }
       l += (rs[0].x + rs[1].x) + (rs[0].y + rs[1].y);
       warp_arrive(p_ready(x), lane);
       ++kept;
