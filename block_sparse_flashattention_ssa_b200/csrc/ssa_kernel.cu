@@ -23,6 +23,10 @@
 // commit tracks every earlier MMA of the thread, so when S_X(j+1) is reported
 // complete every MMA into O_X issued before it has completed too (the softmax
 // may rescale O_X and overwrite the P_X columns without a further wait).
+// A block's skip decision reaches the issuer as a tagged word in shared
+// memory that it polls with acquire loads (the producer, which decides the V
+// loads, waits on a barrier instead): on the issuing thread a barrier wait
+// stalls longer behind its in-flight MMAs than a load does.
 // The two softmax groups run out of phase: one group's exponentials overlap
 // the MMAs of the other.
 // TMEM (512 columns): S_A [0,128) S_B [128,256) O_A [256,256+D)
@@ -103,7 +107,7 @@ struct Ctl {
   uint64_t o_final, drain;
   uint32_t tmem_base;
   int abort_flag;
-  int dec[kQBlocks][kDecRing];
+  int dec[kQBlocks][kDecRing];  // decision of tile j in slot j % kDecRing: ((j + 1) << 1) | skip
   float red[kQBlocks][2][4];
   float cal_red[kQBlocks][2][kCalWindow][4];  // calibration: each warp's vote per tile, double-buffered windows
   int seq, qb_a, has_b, S, start, gqb_a, nq_total;
@@ -137,6 +141,26 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
     if ((i & 31u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        atomicOr(&g_status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded poll of a tagged decision word until it carries `tag` (the tile
+// index + 1); returns the word. Same limit and abort protocol as wait_bar.
+__device__ __forceinline__ bool wait_decision(uint32_t addr, int tag, int& word, volatile int* abort_flag) {
+  word = ld_acquire_shared(addr);
+  if ((word >> 1) == tag) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    word = ld_acquire_shared(addr);
+    if ((word >> 1) == tag) return true;
+    if ((i & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
         *abort_flag = 1;
         atomicOr(&g_status, kStatusTimeout);
         return false;
@@ -257,6 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(o_final, 1);
     mbar_init(smem_u32(&ctl.drain), 1);
     ctl.abort_flag = 0;
+    for (int x = 0; x < kQBlocks; ++x)
+      for (int i = 0; i < kDecRing; ++i) ctl.dec[x][i] = 0;  // tag 0: no tile yet
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -305,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
-            need_v = reinterpret_cast<volatile int*>(ctl.dec[x])[j % kDecRing] == 0;
+            need_v = (reinterpret_cast<volatile int*>(ctl.dec[x])[j % kDecRing] & 1) == 0;
           }
           if (!ok) break;
         }
@@ -390,8 +416,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           bool skip = false;
           if (MODE == kSkip) {
             // The decision also says every warp of the group has read S_X(j).
-            if (!(ok = wait_bar(dec_ready(x, j % kDecRing), (j / kDecRing) & 1, abort_flag))) break;
-            skip = reinterpret_cast<volatile int*>(ctl.dec[x])[j % kDecRing] != 0;
+            int word;
+            if (!(ok = wait_decision(smem_u32(&ctl.dec[x][j % kDecRing]), j + 1, word, abort_flag))) break;
+            skip = (word & 1) != 0;
           }
           if (!skip) {
             if (!(ok = wait_bar(p_ready(x), kept[x] & 1, abort_flag))) break;
@@ -514,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (MODE == kSkip && gt == 0) {
-          reinterpret_cast<volatile int*>(ctl.dec[x])[j % kDecRing] = skip ? 1 : 0;
+          st_release_shared(smem_u32(&ctl.dec[x][j % kDecRing]), ((j + 1) << 1) | (skip ? 1 : 0));
           mbar_arrive(dec_ready(x, j % kDecRing));
         }
       }
