@@ -37,6 +37,13 @@ HEADLINE_TARGET = 0.7
 TARGETS = [0.5, 0.7, 0.9]
 TILE = 128
 WORKLOADS = {"wan14b": "WAN14B", "wan5b": "WAN5B", "tiny": "TINY", "varlen": "VARLEN"}
+# threshold_scale_factor values each workload is specified at (--tsf-sweep).
+# The S = 75,600 shape takes tsf = a*exp(b*s) with the pages' example
+# coefficients a = 0.0003, b = 7.5 at s = 0.5 / 0.7 / 0.9.
+PAGE_EXAMPLE_A, PAGE_EXAMPLE_B = 0.0003, 7.5
+SWEEPS = {"tiny": [0.0, 100.0, 1000.0], "wan5b": [0.0, 1e2, 1e3, 5e3, 2e4],
+          "wan14b": [0.0] + [PAGE_EXAMPLE_A * math.exp(PAGE_EXAMPLE_B * s) for s in TARGETS],
+          "varlen": [0.0, 5000.0]}
 
 
 def peaks():
@@ -503,6 +510,44 @@ def run_calib_sweep(args):
                       "targets_on_benchmark_input": achieved, "runs": runs}), flush=True)
 
 
+def run_tsf_sweep(args):
+    """The forward at each threshold the workload is specified at: time
+    (median of CUDA-event timings), skip ratio and speedup over tsf = 0."""
+    import torch
+
+    import block_sparse_flashattention_ssa_b200 as ssa
+    import synth
+
+    dev = torch.device("cuda", 0)
+    w = getattr(synth, WORKLOADS[args.workload])
+    q, k, v = synth.generate(w)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    dcu = torch.from_numpy(w.cu_seqlens).to(dev)
+    skip = torch.zeros((w.H, ssa.num_qblocks(w.cu_seqlens)), dtype=torch.int32, device=dev)
+    out = torch.empty_like(dq)
+    stream = torch.cuda.current_stream()
+    tiles = tiles_of(w.seqlens, w.H)
+    reps = 5 if w.dense_flop() > 1e14 else 20
+    rows = []
+    for t in SWEEPS[args.workload]:
+        call = lambda t=t: ssa.fwd(dq, dk, dv, dcu, w.max_seqlen, t, out=out, skip_counter=skip)
+        for _ in range(3):
+            call()
+        ms = statistics.median(time_fwd(ssa, call, reps, stream))
+        ssa.check_device()
+        r = float(skip.sum().item()) / tiles
+        rows.append(dict(tsf=t, ms=ms, skip_ratio=r, dense_eq_tflops=w.dense_flop() / ms / 1e9,
+                         effective_tflops=algorithmic_flop(w.seqlens, w.D, w.H, r) / ms / 1e9))
+    for r in rows:
+        r["speedup_vs_dense"] = rows[0]["ms"] / r["ms"]
+    qkv = 3 * w.total_tokens * w.H * w.D * 2
+    print(json.dumps({"metric": "skip-softmax forward at the specified thresholds",
+                      "config": {"workload": w.name, "reps": reps, "qkv_bytes": qkv,
+                                 "l2": "inputs larger than L2" if qkv > 126e6 else "inputs fit in L2"},
+                      "rows": rows}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -515,6 +560,8 @@ def main():
                     help="problem shape (the default is the benchmark workload; the others serve profiling)")
     ap.add_argument("--calib-sweep", action="store_true",
                     help="calibration over 4 seeds x 4 amplitudes, fit, and achieved vs target sparsity")
+    ap.add_argument("--tsf-sweep", action="store_true",
+                    help="time the forward at each threshold the workload is specified at")
     ap.add_argument("--tsf", type=float, default=None,
                     help="fixed threshold_scale_factor: skip calibration and the side rows")
     args = ap.parse_args()
@@ -522,6 +569,8 @@ def main():
         run_reference(args)
     elif args.calib_sweep:
         run_calib_sweep(args)
+    elif args.tsf_sweep:
+        run_tsf_sweep(args)
     else:
         run_ours(args)
 

@@ -30,8 +30,11 @@
 // The two softmax groups run out of phase: one group's exponentials overlap
 // the MMAs of the other.
 // TMEM (512 columns): S_A [0,128) S_B [128,256) O_A [256,256+D)
-// O_B [384,384+D); P_X occupies the first 64 columns of S_X as packed bf16
-// pairs.
+// O_B [384,384+D); P_X is written over S_X as packed bf16 pairs: in the dense
+// and calibration kernels to columns [0,64) in kv order, in the skipping
+// kernel kv [0,64) to columns [0,32) and kv [64,128) to [64,96), so the upper
+// half can be stored as soon as it is computed (its S columns have been read)
+// while the lower half of S is still being read back.
 //
 // Every wait on an mbarrier is bounded in time; when one runs out the CTA
 // records SSA_ERR_TIMEOUT in the device status word, the other roles see the
@@ -381,7 +384,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(s_full(x));
       };
-      // O_X += P_X V from the TMEM copy of P_X and V stage vs.
+      // O_X += P_X V from the TMEM copy of P_X and V stage vs. The skipping
+      // kernel keeps P of kv [64,128) at columns [64,96) of S_X.
       auto issue_pv = [&](int x, int vs, bool accumulate) {
         const uint32_t p_tmem = tmem + col_S(x);
         const uint32_t v_s = smem_u32(smem + L::kV + vs * L::kVTileBytes);
@@ -389,7 +393,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int ks = 0; ks < kBN / 16; ++ks) {
           // V is MN-major (d contiguous): 16 kv rows = 2 KB per k step; the
           // second 64-column chunk of d sits one 16 KB chunk further (LBO).
-          mma_ts(tmem + col_O(x), p_tmem + ks * 8, smem_desc_sw128(v_s + ks * 16 * 128, L::kChunkBytes, 1024),
+          const uint32_t p_col = ks * 8 + ((MODE == kSkip && ks >= kBN / 32) ? 32 : 0);
+          mma_ts(tmem + col_O(x), p_tmem + p_col, smem_desc_sw128(v_s + ks * 16 * 128, L::kChunkBytes, 1024),
                  idesc_pv, (accumulate || ks > 0) ? 1u : 0u);
         }
       };
@@ -574,9 +579,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       uint32_t lo[64];
       tmem_ld_x64_async(lane_base + col_s, lo);  // lands while the upper half is exponentiated
-      // Packed P: [0,32) from S columns [0,64), [32,64) from [64,128). The
-      // dense and calibration kernels store it with one 64-column store; the
-      // skipping kernel, which has less register room, with two.
+      // Packed P: bf16 pairs of consecutive kv columns. The dense and
+      // calibration kernels keep all 64 pairs in registers and store them to
+      // columns [0,64) at once; the skipping kernel, which has less register
+      // room, stores the upper half's pairs to columns [64,96) right away.
       uint32_t pk[64];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -585,6 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         rs[i & 1] = fadd2(rs[i & 1], e);
         pk[32 + i] = pack_bf16x2(e.x, e.y);
       }
+      if (MODE == kSkip) tmem_st_x32(lane_base + col_s + 64, reinterpret_cast<const uint32_t(&)[32]>(pk[32]));
       tmem_wait_ld_tied(lo);
       if (valid < 64) {
 #pragma unroll
@@ -599,12 +606,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         pk[i] = pack_bf16x2(e.x, e.y);
       }
       // Both halves of S_X are in registers by now: P_X may overwrite them.
-      if (MODE == kSkip) {
+      if (MODE == kSkip)
         tmem_st_x32(lane_base + col_s, reinterpret_cast<const uint32_t(&)[32]>(pk[0]));
-        tmem_st_x32(lane_base + col_s + 32, reinterpret_cast<const uint32_t(&)[32]>(pk[32]));
-      } else {
+      else
         tmem_st_x64(lane_base + col_s, pk);
-      }
       l += (rs[0].x + rs[1].x) + (rs[0].y + rs[1].y);
       warp_arrive(p_ready(x), lane);
       ++kept;

@@ -63,3 +63,16 @@ def test_peaks_prefer_the_measured_file(tmp_path, monkeypatch):
     assert bench.peaks() == (1625.5, 1389.3, 6558, "measured")
     os.remove(os.path.join(root, "MEASURED_PEAKS.json"))
     assert bench.peaks()[3] == "fallback"
+
+
+def test_threshold_sweeps_are_the_specified_values():
+    """--tsf-sweep times the forward at the thresholds each workload is
+    specified at; the S = 75,600 ones come from the pages' example formula
+    tsf = 0.0003 * exp(7.5 * s) at s = 0.5 / 0.7 / 0.9."""
+    assert bench.SWEEPS["tiny"] == [0.0, 100.0, 1000.0]
+    assert bench.SWEEPS["wan5b"] == [0.0, 1e2, 1e3, 5e3, 2e4]
+    assert bench.SWEEPS["varlen"] == [0.0, 5000.0]
+    got = bench.SWEEPS["wan14b"]
+    assert got[0] == 0.0
+    for g, want in zip(got[1:], [0.012756, 0.057170, 0.256218]):
+        assert abs(g - want) < 1e-6
