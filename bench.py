@@ -497,16 +497,25 @@ def run_calib_sweep(args):
     dq, dk, dv, dcu, w = first
     skip = torch.zeros((w.H, ssa.num_qblocks(w.cu_seqlens)), dtype=torch.int32, device=dev)
     achieved = {}
-    for s_t in TARGETS:
-        tsf = ssa.resolve(a, b, s_t)
-        ssa.fwd(dq, dk, dv, dcu, w.max_seqlen, tsf, skip_counter=skip)
+    stream = torch.cuda.current_stream()
+    dense_ms = None
+    for s_t in [0.0] + TARGETS:  # 0.0: the same kernel with skipping off
+        tsf = ssa.resolve(a, b, s_t) if s_t > 0 else 0.0
+        call = lambda t=tsf: ssa.fwd(dq, dk, dv, dcu, w.max_seqlen, t, skip_counter=skip)
+        call()
+        ms = statistics.median(time_fwd(ssa, call, 5, stream))
         ssa.check_device()
-        achieved[str(s_t)] = {"tsf": tsf, "achieved_sparsity": float(skip.sum().item()) / tiles}
+        if s_t == 0.0:
+            dense_ms = ms
+            continue
+        achieved[str(s_t)] = {"tsf": tsf, "achieved_sparsity": float(skip.sum().item()) / tiles, "ms": ms,
+                              "speedup_vs_dense": dense_ms / ms}
     print(json.dumps({"metric": "calibration sweep: fit of threshold_scale_factor = a*exp(b*s)",
                       "config": {"workload": base.name, "seeds": synth.CALIB_SEEDS, "amps": synth.CALIB_AMPS,
                                  "thresholds": lams},
                       "fit": {"a": a, "b": b, "s_min": smin, "s_max": smax, "points": len(pts_s)},
                       "calib_ms_mean": statistics.mean(r["calib_ms"] for r in runs),
+                      "dense_ms_on_benchmark_input": dense_ms,
                       "targets_on_benchmark_input": achieved, "runs": runs}), flush=True)
 
 
