@@ -133,3 +133,18 @@ def test_fp8_entry_points_validate_on_the_host(ssa):
     assert qz(mis, fake, 16, 1.0) == ssa.SSA_ERR_UNSUPPORTED
     assert qz(fake, ctypes.c_void_p(0x10004), 16, 1.0) == ssa.SSA_ERR_UNSUPPORTED
     assert qz(fake, fake, 0, 1.0) == ssa.SSA_OK
+
+
+def test_package_refuses_to_import_without_its_library(tmp_path):
+    """No CPU fallback: a copy of the package without libssa.so fails at
+    import with a message naming the missing library."""
+    import shutil
+    import sys
+
+    src = os.path.join(ROOT, "block_sparse_flashattention_ssa_b200")
+    shutil.copytree(src, tmp_path / "block_sparse_flashattention_ssa_b200",
+                    ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    r = subprocess.run([sys.executable, "-c", "import block_sparse_flashattention_ssa_b200"], cwd=str(tmp_path),
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "libssa.so is not built" in r.stderr
