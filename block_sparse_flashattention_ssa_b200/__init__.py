@@ -12,6 +12,7 @@ Entry points (same names as the C ABI, without the ``ssa_`` prefix):
   fwd_fp8      the forward with E4M3 Q and K (per-tensor descales)
   quantize_fp8 bf16 -> E4M3 per-tensor quantisation for fwd_fp8
   calibrate    dense attention + skip counts at N thresholds at once
+               (optionally with the per-tile statistic, ``ssa_calibrate_ex``)
   calibrate_fp8  the same with E4M3 Q and K
   resolve      threshold_scale_factor = a * exp(b * target_sparsity)
   fit_logspace log-space least-squares fit of (a, b)
@@ -21,7 +22,6 @@ Entry points (same names as the C ABI, without the ``ssa_`` prefix):
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 
 import numpy as np
@@ -54,17 +54,20 @@ def _load():
     L = ctypes.CDLL(_SO)
     vp, i32, f32, f64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_double
     L.ssa_fwd.restype = i32
-    L.ssa_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp]
+    L.ssa_fwd.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, i32, vp]
     L.ssa_fwd_ex.restype = i32
-    L.ssa_fwd_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, vp, vp, vp]
+    L.ssa_fwd_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp, i32, vp, vp, vp]
     L.ssa_fwd_fp8.restype = i32
-    L.ssa_fwd_fp8.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32, f32, vp, vp, vp, vp, vp]
+    L.ssa_fwd_fp8.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32, f32, vp, vp, i32, vp, vp, vp]
     L.ssa_calibrate_fp8.restype = i32
-    L.ssa_calibrate_fp8.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32, vp, i32, vp, vp, vp]
+    L.ssa_calibrate_fp8.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32, vp, i32, vp, vp, i32,
+                                    vp]
     L.ssa_quantize_fp8.restype = i32
     L.ssa_quantize_fp8.argtypes = [vp, vp, ctypes.c_int64, f32, vp]
     L.ssa_calibrate.restype = i32
-    L.ssa_calibrate.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32, vp, vp, vp]
+    L.ssa_calibrate.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32, vp, vp, i32, vp]
+    L.ssa_calibrate_ex.restype = i32
+    L.ssa_calibrate_ex.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, vp, i32, vp, vp, i32, vp, vp]
     L.ssa_resolve.restype = f64
     L.ssa_resolve.argtypes = [f64, f64, f64]
     L.ssa_fit_logspace.restype = i32
@@ -156,10 +159,30 @@ def _check_attention_args(q, k, v, cu_seqlens, out, qk_dtype):
     return dev
 
 
-def _check_per_unit(t, name, dtype, dev, H):
-    _require(t, name, dtype, dev, allow_none=True)
-    if t is not None and (t.dim() < 2 or t.shape[0] != H):
-        raise ValueError(f"{name} must be [num_heads, num_qblocks, ...] with num_heads = {H}")
+def _per_unit_qblocks(dev, H, total, batch, outputs) -> int:
+    """Check the per-unit outputs ``(tensor, name, dtypes, inner_shape)``:
+    each must be [H, Q, *inner_shape] on ``dev``, all with the same Q, and Q
+    no larger than any batch of ``total`` tokens can have. Returns that Q
+    (-1 when every output is None). The library counts the q-blocks again
+    from the device copy of cu_seqlens and writes nothing when they differ,
+    so a wrong Q cannot overrun a buffer either way."""
+    q_dim = None
+    for t, name, dtype, inner in outputs:
+        _require(t, name, dtype, dev, allow_none=True)
+        if t is None:
+            continue
+        if t.dim() != 2 + len(inner) or t.shape[0] != H or tuple(t.shape[2:]) != tuple(inner):
+            want = ", ".join([str(H), "num_qblocks"] + [str(i) for i in inner])
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected [{want}]")
+        if q_dim is None:
+            q_dim = int(t.shape[1])
+        elif int(t.shape[1]) != q_dim:
+            raise ValueError(f"{name} has {t.shape[1]} q-blocks, another per-unit output {q_dim}")
+    if q_dim is None:
+        return -1
+    if q_dim > (total + TILE - 1) // TILE + batch:
+        raise ValueError(f"{q_dim} q-blocks is more than {total} tokens in {batch} sequences can have")
+    return q_dim
 
 
 def num_qblocks(cu_seqlens) -> int:
@@ -184,14 +207,13 @@ def fwd(q, k, v, cu_seqlens, max_seqlen: int, threshold_scale_factor: float = 0.
 
     total, H, D = _shape(q)
     dev = _check_attention_args(q, k, v, cu_seqlens, out, torch.bfloat16)
-    _check_per_unit(skip_counter, "skip_counter", torch.int32, dev, H)
-    _check_per_unit(decision_bitmap, "decision_bitmap", (torch.int32, torch.uint32), dev, H)
-    _check_per_unit(tile_stat, "tile_stat", torch.float32, dev, H)
+    batch = cu_seqlens.numel() - 1
+    nq = _per_unit_qblocks(dev, H, total, batch, _forward_outputs(skip_counter, decision_bitmap, tile_stat,
+                                                                  max_seqlen))
     if out is None:
         out = torch.empty_like(q)
-    batch = cu_seqlens.numel() - 1
     args = [_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D,
-            float(softmax_scale), float(threshold_scale_factor), _ptr(out), _ptr(skip_counter)]
+            float(softmax_scale), float(threshold_scale_factor), _ptr(out), _ptr(skip_counter), nq]
     if decision_bitmap is not None or tile_stat is not None:
         rc = _lib.ssa_fwd_ex(*args, _ptr(decision_bitmap), _ptr(tile_stat), _stream_handle(stream))
         _check(rc, "ssa_fwd_ex")
@@ -209,15 +231,14 @@ def fwd_fp8(q8, k8, v, cu_seqlens, max_seqlen: int, q_descale: float, k_descale:
 
     total, H, D = _shape(q8)
     dev = _check_attention_args(q8, k8, v, cu_seqlens, out, torch.uint8)
-    _check_per_unit(skip_counter, "skip_counter", torch.int32, dev, H)
-    _check_per_unit(decision_bitmap, "decision_bitmap", (torch.int32, torch.uint32), dev, H)
-    _check_per_unit(tile_stat, "tile_stat", torch.float32, dev, H)
+    batch = cu_seqlens.numel() - 1
+    nq = _per_unit_qblocks(dev, H, total, batch, _forward_outputs(skip_counter, decision_bitmap, tile_stat,
+                                                                  max_seqlen))
     if out is None:
         out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
-    batch = cu_seqlens.numel() - 1
     rc = _lib.ssa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D,
                           float(softmax_scale), float(q_descale), float(k_descale), float(threshold_scale_factor),
-                          _ptr(out), _ptr(skip_counter), _ptr(decision_bitmap), _ptr(tile_stat),
+                          _ptr(out), _ptr(skip_counter), nq, _ptr(decision_bitmap), _ptr(tile_stat),
                           _stream_handle(stream))
     _check(rc, "ssa_fwd_fp8")
     return out
@@ -239,28 +260,31 @@ def quantize_fp8(x, inv_scale: float, out=None, stream=None):
 
 
 def calibrate(q, k, v, cu_seqlens, max_seqlen: int, thresholds, softmax_scale: float = 0.0, out=None, counts=None,
-              stream=None):
+              tile_stat=None, stream=None):
     """Dense attention plus, per (head, q-block) unit, the number of KV tiles
     that would be skipped at each raw lambda in ``thresholds``. Returns
-    (out, counts[H, Q, N])."""
+    (out, counts[H, Q, N]). Passing ``tile_stat`` (float32 [H, Q, T],
+    caller-allocated) selects ``ssa_calibrate_ex``, which also writes every
+    tile's statistic d_j. Without ``counts`` the q-block count is read from a
+    host copy of cu_seqlens (a synchronisation)."""
     import torch
 
     total, H, D = _shape(q)
     dev = _check_attention_args(q, k, v, cu_seqlens, out, torch.bfloat16)
-    _check_per_unit(counts, "counts", torch.int32, dev, H)
     th = np.ascontiguousarray(thresholds, dtype=np.float32)
-    if counts is not None and (counts.dim() != 3 or counts.shape[2] != len(th)):
-        raise ValueError("counts must be [num_heads, num_qblocks, n_thresholds]")
+    batch = cu_seqlens.numel() - 1
+    if counts is None:
+        counts = torch.empty((H, num_qblocks(cu_seqlens), len(th)), dtype=torch.int32, device=dev)
+    nq = _per_unit_qblocks(dev, H, total, batch, [(counts, "counts", torch.int32, (len(th),)),
+                                                   (tile_stat, "tile_stat", torch.float32, (max_tiles(max_seqlen),))])
     if out is None:
         out = torch.empty_like(q)
-    if counts is None:
-        Q = num_qblocks(cu_seqlens)
-        counts = torch.empty((H, Q, len(th)), dtype=torch.int32, device=q.device)
-    batch = cu_seqlens.numel() - 1
-    rc = _lib.ssa_calibrate(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D,
-                            float(softmax_scale), th.ctypes.data, len(th), _ptr(out), _ptr(counts),
-                            _stream_handle(stream))
-    _check(rc, "ssa_calibrate")
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D, float(softmax_scale),
+            th.ctypes.data, len(th), _ptr(out), _ptr(counts), nq]
+    if tile_stat is not None:
+        _check(_lib.ssa_calibrate_ex(*args, _ptr(tile_stat), _stream_handle(stream)), "ssa_calibrate_ex")
+    else:
+        _check(_lib.ssa_calibrate(*args, _stream_handle(stream)), "ssa_calibrate")
     return out, counts
 
 
@@ -271,18 +295,16 @@ def calibrate_fp8(q8, k8, v, cu_seqlens, max_seqlen: int, q_descale: float, k_de
 
     total, H, D = _shape(q8)
     dev = _check_attention_args(q8, k8, v, cu_seqlens, out, torch.uint8)
-    _check_per_unit(counts, "counts", torch.int32, dev, H)
     th = np.ascontiguousarray(thresholds, dtype=np.float32)
-    if counts is not None and (counts.dim() != 3 or counts.shape[2] != len(th)):
-        raise ValueError("counts must be [num_heads, num_qblocks, n_thresholds]")
-    if out is None:
-        out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    batch = cu_seqlens.numel() - 1
     if counts is None:
         counts = torch.empty((H, num_qblocks(cu_seqlens), len(th)), dtype=torch.int32, device=dev)
-    batch = cu_seqlens.numel() - 1
+    nq = _per_unit_qblocks(dev, H, total, batch, [(counts, "counts", torch.int32, (len(th),))])
+    if out is None:
+        out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
     rc = _lib.ssa_calibrate_fp8(_ptr(q8), _ptr(k8), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D,
                                 float(softmax_scale), float(q_descale), float(k_descale), th.ctypes.data, len(th),
-                                _ptr(out), _ptr(counts), _stream_handle(stream))
+                                _ptr(out), _ptr(counts), nq, _stream_handle(stream))
     _check(rc, "ssa_calibrate_fp8")
     return out, counts
 
@@ -333,8 +355,9 @@ def bitmap_words(max_seqlen: int) -> int:
     return (max_tiles(max_seqlen) + 31) // 32
 
 
-def threshold_log2(threshold_scale_factor: float, s_kv: int) -> float:
-    """Host helper for callers and reports: log2(tsf / S_kv), -inf when tsf <= 0."""
-    if threshold_scale_factor <= 0:
-        return -math.inf
-    return math.log2(threshold_scale_factor / s_kv)
+def _forward_outputs(skip_counter, decision_bitmap, tile_stat, max_seqlen):
+    import torch
+
+    return [(skip_counter, "skip_counter", torch.int32, ()),
+            (decision_bitmap, "decision_bitmap", (torch.int32, torch.uint32), (bitmap_words(max_seqlen),)),
+            (tile_stat, "tile_stat", torch.float32, (max_tiles(max_seqlen),))]

@@ -95,6 +95,7 @@ struct Params {
   uint32_t* bitmap;
   float* tile_stat;
   int batch, total_tokens, num_heads, max_tiles, bitmap_words;
+  int nq_check;  // q-blocks the per-unit outputs are sized for, or -1 when there are none
   float c;    // fp32(softmax_scale * log2 e)
   float tsf;  // threshold_scale_factor (kSkip)
   int n_cal;
@@ -197,6 +198,101 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
+// Maps this CTA (blockIdx.x) to its (sequence, pair of query blocks) and
+// validates cu_seqlens; run by the whole of warp 0. For batches of up to 32
+// sequences the pairs are numbered longest sequence first (ties by index), so
+// the units with the longest KV walks start first and short ones fill the end
+// of the grid; larger batches keep sequence order. Either way the per-unit
+// outputs are indexed by the global q-block in sequence order. A CTA past the
+// last pair gets ctl.seq = -1, and so does every CTA when the input is
+// inconsistent: cu_seqlens negative, decreasing or past total_tokens, a
+// sequence longer than max_seqlen where the diagnostics are sized from it, or
+// a q-block count other than the one the caller sized its per-unit outputs
+// for (p.nq_check >= 0). Inconsistencies are reported in the status word.
+__device__ void locate_unit(const Params& p, bool need_max, int lane, Ctl& ctl) {
+  const int x = static_cast<int>(blockIdx.x);
+  int seq = -1, qb_a = 0, has_b = 0, start = 0, S = 0, gqb_a = 0, bad = 0, nq_total = 0;
+  if (p.batch <= 32) {
+    const int b = lane;  // one sequence per lane
+    int lo = 0, len = 0, nq = 0, np = 0;
+    if (b < p.batch) {
+      lo = p.cu_seqlens[b];
+      const int hi = p.cu_seqlens[b + 1];
+      len = hi - lo;
+      if (lo < 0 || len < 0 || hi > p.total_tokens) bad = 1;
+      nq = (len + kBM - 1) / kBM;
+      np = (nq + 1) / 2;
+      if (need_max && nq > p.max_tiles) bad = 1;
+    }
+    bad = __any_sync(kFull, bad) ? 1 : 0;
+    int q_off = nq;  // inclusive prefix sum of q-blocks in sequence order
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(kFull, q_off, o);
+      if (lane >= o) q_off += t;
+    }
+    nq_total = __shfl_sync(kFull, q_off, 31);
+    q_off -= nq;
+    int p_off = 0;  // first pair of sequence b in longest-first order
+    for (int o = 0; o < p.batch; ++o) {
+      const int len_o = __shfl_sync(kFull, len, o), np_o = __shfl_sync(kFull, np, o);
+      if (len_o > len || (len_o == len && o < b)) p_off += np_o;
+    }
+    const unsigned who = __ballot_sync(kFull, b < p.batch && x >= p_off && x < p_off + np);
+    if (who) {
+      const int src = __ffs(static_cast<int>(who)) - 1;
+      const int pair = __shfl_sync(kFull, x - p_off, src);
+      const int nq_s = __shfl_sync(kFull, nq, src);
+      seq = src;
+      qb_a = 2 * pair;
+      has_b = qb_a + 1 < nq_s ? 1 : 0;
+      gqb_a = __shfl_sync(kFull, q_off, src) + qb_a;
+      start = __shfl_sync(kFull, lo, src);
+      S = __shfl_sync(kFull, len, src);
+    }
+  } else if (lane == 0) {
+    int accp = 0;
+    int prev = p.cu_seqlens[0];
+    if (prev < 0) bad = 1;
+    for (int b = 0; b < p.batch && !bad; ++b) {
+      const int nxt = p.cu_seqlens[b + 1];
+      const int len = nxt - prev;
+      if (len < 0 || nxt > p.total_tokens) {
+        bad = 1;
+        break;
+      }
+      const int nq = (len + kBM - 1) / kBM;
+      const int np = (nq + 1) / 2;
+      if (need_max && nq > p.max_tiles) bad = 1;
+      if (seq < 0 && x < accp + np) {
+        seq = b;
+        qb_a = 2 * (x - accp);
+        has_b = qb_a + 1 < nq ? 1 : 0;
+        gqb_a = nq_total + qb_a;
+        start = prev;
+        S = len;
+      }
+      nq_total += nq;
+      accp += np;
+      prev = nxt;
+    }
+  }
+  if (lane == 0) {
+    if (!bad && p.nq_check >= 0 && nq_total != p.nq_check) bad = 1;
+    if (bad) {
+      if (x == 0) atomicOr(&g_status, kStatusDeviceArg);
+      seq = -1;
+    }
+    ctl.seq = seq;
+    ctl.qb_a = qb_a;
+    ctl.has_b = has_b;
+    ctl.S = S;
+    ctl.start = start;
+    ctl.gqb_a = gqb_a;
+    ctl.nq_total = nq_total;
+  }
+}
+
 template <int D, int MODE, bool EX, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     ssa_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -209,45 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int head = blockIdx.y;
 
-  // Locate this CTA's (sequence, pair of q-blocks) and validate cu_seqlens.
-  if (threadIdx.x == 0) {
-    int accq = 0, accp = 0, seq = -1, qb_a = 0, has_b = 0, start = 0, S = 0, gqb_a = 0, bad = 0;
-    int prev = p.cu_seqlens[0];
-    if (prev < 0) bad = 1;
-    for (int b = 0; b < p.batch && !bad; ++b) {
-      const int nxt = p.cu_seqlens[b + 1];
-      const int len = nxt - prev;
-      if (len < 0 || nxt > p.total_tokens) {
-        bad = 1;
-        break;
-      }
-      const int nq = (len + kBM - 1) / kBM;
-      const int np = (nq + 1) / 2;
-      if (seq < 0 && static_cast<int>(blockIdx.x) < accp + np) {
-        seq = b;
-        qb_a = 2 * (static_cast<int>(blockIdx.x) - accp);
-        has_b = qb_a + 1 < nq ? 1 : 0;
-        gqb_a = accq + qb_a;
-        start = prev;
-        S = len;
-      }
-      accq += nq;
-      accp += np;
-      prev = nxt;
-    }
-    if (!bad && seq >= 0 && (EX && (S + kBN - 1) / kBN > p.max_tiles)) bad = 1;
-    if (bad) {
-      if (blockIdx.x == 0) atomicOr(&g_status, kStatusDeviceArg);
-      seq = -1;
-    }
-    ctl.seq = seq;
-    ctl.qb_a = qb_a;
-    ctl.has_b = has_b;
-    ctl.S = S;
-    ctl.start = start;
-    ctl.gqb_a = gqb_a;
-    ctl.nq_total = accq;
-  }
+  if (warp == 0) locate_unit(p, EX, lane, ctl);
   __syncthreads();
   if (ctl.seq < 0) return;  // uniform: no unit for this CTA (or bad input)
 
@@ -520,6 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (i <= slot) {
             volatile float* r = ctl.cal_red[x][win & 1][i];
             const float d = fmaxf(fmaxf(r[0], r[1]), fmaxf(r[2], r[3]));
+            if (EX && gt < kCalWindow && p.tile_stat) p.tile_stat[unit * p.max_tiles + win * kCalWindow + i] = d;
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
               const int k = (gt >> 4) + 8 * m;
@@ -681,6 +740,9 @@ __global__ void wait_timeout_check_kernel(uint64_t limit_ns, int* result) {
   result[2] = static_cast<int>((globaltimer_ns() - t0) / 1000);  // microseconds waited
 }
 
+// Clears the given bits of the status word atomically (ssa_get_error).
+__global__ void status_clear_kernel(int bits) { atomicAnd(&g_status, ~bits); }
+
 // ----------------------------------------------------------------- host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -770,6 +832,7 @@ Params base_params(const Call& a) {
   p.num_heads = a.H;
   p.max_tiles = (a.max_seqlen + kBN - 1) / kBN;
   p.bitmap_words = (p.max_tiles + 31) / 32;
+  p.nq_check = -1;
   double scale = a.softmax_scale > 0.f ? static_cast<double>(a.softmax_scale) : 1.0 / std::sqrt(static_cast<double>(a.D));
   if (a.f8) scale = scale * a.qk_descale;  // E4M3 codes carry the per-tensor scales of Q and K
   p.c = static_cast<float>(scale * 1.4426950408889634073599246810019);
@@ -833,14 +896,17 @@ __global__ void quantize_e4m3_kernel(const __nv_bfloat16* __restrict__ x, uint8_
   }
 }
 
-int fwd_impl(const Call& a, float tsf, int32_t* skip_counter, uint32_t* bitmap, float* tile_stat) {
+int fwd_impl(const Call& a, float tsf, int32_t* skip_counter, int num_qblocks, uint32_t* bitmap, float* tile_stat) {
   int rc = validate(a);
   if (rc != SSA_OK) return rc;
   if (std::isnan(tsf) || std::isinf(tsf)) return SSA_ERR_INVALID_ARG;
   if ((bitmap || tile_stat) && a.max_seqlen < 1) return SSA_ERR_INVALID_ARG;
+  const bool per_unit = skip_counter || bitmap || tile_stat;
+  if (per_unit && num_qblocks < 0) return SSA_ERR_INVALID_ARG;
   if (a.total_tokens == 0) return SSA_OK;
   if ((rc = check_device_pointers({skip_counter, bitmap, tile_stat})) != SSA_OK) return rc;
   Params p = base_params(a);
+  p.nq_check = per_unit ? num_qblocks : -1;
   p.skip_counter = skip_counter;
   p.bitmap = bitmap;
   p.tile_stat = tile_stat;
@@ -858,14 +924,15 @@ using namespace ssa;
 extern "C" int ssa_fwd_fp8(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
                            int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
                            float q_descale, float k_descale, float threshold_scale_factor, void* out,
-                           int32_t* skip_counter, uint32_t* decision_bitmap, float* tile_stat, void* stream) {
+                           int32_t* skip_counter, int num_qblocks, uint32_t* decision_bitmap, float* tile_stat,
+                           void* stream) {
   Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
          static_cast<cudaStream_t>(stream)};
   if (!(q_descale > 0.f) || !(k_descale > 0.f) || std::isinf(q_descale) || std::isinf(k_descale))
     return SSA_ERR_INVALID_ARG;
   a.f8 = true;
   a.qk_descale = static_cast<double>(q_descale) * static_cast<double>(k_descale);
-  return fwd_impl(a, threshold_scale_factor, skip_counter, decision_bitmap, tile_stat);
+  return fwd_impl(a, threshold_scale_factor, skip_counter, num_qblocks, decision_bitmap, tile_stat);
 }
 
 extern "C" int ssa_quantize_fp8(const void* x, void* y, int64_t n, float inv_scale, void* stream) {
@@ -886,59 +953,75 @@ extern "C" int ssa_quantize_fp8(const void* x, void* y, int64_t n, float inv_sca
 
 extern "C" int ssa_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
                        int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
-                       float threshold_scale_factor, void* out, int32_t* skip_counter, void* stream) {
+                       float threshold_scale_factor, void* out, int32_t* skip_counter, int num_qblocks,
+                       void* stream) {
   const Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
                static_cast<cudaStream_t>(stream)};
-  return fwd_impl(a, threshold_scale_factor, skip_counter, nullptr, nullptr);
+  return fwd_impl(a, threshold_scale_factor, skip_counter, num_qblocks, nullptr, nullptr);
 }
 
 extern "C" int ssa_fwd_ex(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
                           int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
-                          float threshold_scale_factor, void* out, int32_t* skip_counter, uint32_t* decision_bitmap,
-                          float* tile_stat, void* stream) {
+                          float threshold_scale_factor, void* out, int32_t* skip_counter, int num_qblocks,
+                          uint32_t* decision_bitmap, float* tile_stat, void* stream) {
   const Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
                static_cast<cudaStream_t>(stream)};
-  return fwd_impl(a, threshold_scale_factor, skip_counter, decision_bitmap, tile_stat);
+  return fwd_impl(a, threshold_scale_factor, skip_counter, num_qblocks, decision_bitmap, tile_stat);
 }
 
 namespace ssa {
 namespace {
-int calibrate_impl(const Call& a, const float* thresholds, int n_thresholds, int32_t* counts) {
+int calibrate_impl(const Call& a, const float* thresholds, int n_thresholds, int32_t* counts, int num_qblocks,
+                   float* tile_stat) {
   int rc = validate(a);
   if (rc != SSA_OK) return rc;
-  if (!thresholds || !counts || n_thresholds < 1 || n_thresholds > SSA_MAX_THRESHOLDS) return SSA_ERR_INVALID_ARG;
+  if (!thresholds || !counts || n_thresholds < 1 || n_thresholds > SSA_MAX_THRESHOLDS || num_qblocks < 0)
+    return SSA_ERR_INVALID_ARG;
   for (int i = 0; i < n_thresholds; ++i)
     if (!(thresholds[i] > 0.f) || std::isinf(thresholds[i])) return SSA_ERR_INVALID_ARG;
+  if (tile_stat && a.max_seqlen < 1) return SSA_ERR_INVALID_ARG;
   if (a.total_tokens == 0) return SSA_OK;
-  if ((rc = check_device_pointers({counts})) != SSA_OK) return rc;
+  if ((rc = check_device_pointers({counts, tile_stat})) != SSA_OK) return rc;
   Params p = base_params(a);
+  p.nq_check = num_qblocks;
   p.counts = counts;
+  p.tile_stat = tile_stat;
   p.n_cal = n_thresholds;
   for (int i = 0; i < n_thresholds; ++i) p.Lcal[i] = static_cast<float>(std::log2(static_cast<double>(thresholds[i])));
-  return dispatch_d<kCalib, false>(a, p);
+  return tile_stat ? dispatch_d<kCalib, true>(a, p) : dispatch_d<kCalib, false>(a, p);
 }
 }  // namespace
 }  // namespace ssa
 
 extern "C" int ssa_calibrate(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
                              int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
-                             const float* thresholds, int n_thresholds, void* out, int32_t* counts, void* stream) {
+                             const float* thresholds, int n_thresholds, void* out, int32_t* counts, int num_qblocks,
+                             void* stream) {
   const Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
                static_cast<cudaStream_t>(stream)};
-  return calibrate_impl(a, thresholds, n_thresholds, counts);
+  return calibrate_impl(a, thresholds, n_thresholds, counts, num_qblocks, nullptr);
+}
+
+extern "C" int ssa_calibrate_ex(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                                int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                                const float* thresholds, int n_thresholds, void* out, int32_t* counts,
+                                int num_qblocks, float* tile_stat, void* stream) {
+  const Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
+               static_cast<cudaStream_t>(stream)};
+  return calibrate_impl(a, thresholds, n_thresholds, counts, num_qblocks, tile_stat);
 }
 
 extern "C" int ssa_calibrate_fp8(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
                                  int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
                                  float q_descale, float k_descale, const float* thresholds, int n_thresholds,
-                                 void* out, int32_t* counts, void* stream) {
+                                 void* out, int32_t* counts, int num_qblocks, void* stream) {
   Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
          static_cast<cudaStream_t>(stream)};
   if (!(q_descale > 0.f) || !(k_descale > 0.f) || std::isinf(q_descale) || std::isinf(k_descale))
     return SSA_ERR_INVALID_ARG;
   a.f8 = true;
   a.qk_descale = static_cast<double>(q_descale) * static_cast<double>(k_descale);
-  return calibrate_impl(a, thresholds, n_thresholds, counts);
+  return calibrate_impl(a, thresholds, n_thresholds, counts, num_qblocks, nullptr);
 }
 
 extern "C" const char* ssa_last_cuda_error(void) { return t_last_cuda_error; }
@@ -957,10 +1040,11 @@ extern "C" int ssa_get_error(void* stream) {
   int v = 0;
   e = cudaMemcpyFromSymbol(&v, g_status, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e);
-  if (v != 0) {
-    const int zero = 0;
-    e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
-    if (e != cudaSuccess) return cuda_fail(e);
+  if (v != 0) {  // clear exactly the bits read: a bit another stream sets meanwhile stays for the next call
+    status_clear_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(v);
+    if ((e = cudaGetLastError()) != cudaSuccess || (e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream))) !=
+                                                       cudaSuccess)
+      return cuda_fail(e);
   }
   if (v & kStatusTimeout) return SSA_ERR_TIMEOUT;
   if (v & kStatusDeviceArg) return SSA_ERR_DEVICE_ARG;

@@ -40,8 +40,20 @@
  * aligned. Every pointer documented as a device pointer must be device (or
  * managed) memory of the current device: the entry points check this with
  * cudaPointerGetAttributes before any launch and return SSA_ERR_INVALID_ARG
- * otherwise. Buffer sizes cannot be checked: the caller sizes the per-unit
- * outputs from ssa_num_qblocks().
+ * otherwise.
+ *
+ * Per-unit outputs. The caller sizes them from ssa_num_qblocks() (on a host
+ * copy of cu_seqlens) and passes that count as num_qblocks; their inner
+ * sizes follow from max_seqlen and n_thresholds. The kernels count the
+ * q-blocks again from the device copy of cu_seqlens and, when the counts
+ * differ (or a sequence is longer than max_seqlen where the diagnostics are
+ * sized from it), write nothing at all and record SSA_ERR_DEVICE_ARG, so an
+ * undersized buffer is never overrun. num_qblocks is ignored when no
+ * per-unit output is given; a negative value with one is SSA_ERR_INVALID_ARG.
+ *
+ * Work order. For batches of up to 32 sequences the kernels start the
+ * longest sequence's query blocks first (ties by position in the batch);
+ * results do not depend on the order.
  */
 #ifndef SSA_H_
 #define SSA_H_
@@ -58,7 +70,8 @@ enum {
   SSA_ERR_UNSUPPORTED = -2, /* head_dim not 64/128, misaligned pointer      */
   SSA_ERR_CUDA = -3,        /* a CUDA runtime or launch error               */
   SSA_ERR_TIMEOUT = -4,     /* a device-side wait exceeded its time limit   */
-  SSA_ERR_DEVICE_ARG = -5   /* the kernel found cu_seqlens inconsistent     */
+  SSA_ERR_DEVICE_ARG = -5   /* the kernel found cu_seqlens inconsistent (or
+                               with num_qblocks / max_seqlen); nothing written */
 };
 
 #define SSA_TILE 128          /* Br = Bc = 128                                 */
@@ -77,11 +90,13 @@ enum {
  *                every sequence are written, nothing else is touched
  *   skip_counter device int32 [num_heads][Q] or NULL: tiles skipped per unit
  *                (plain stores, no atomics)
+ *   num_qblocks  Q, the count skip_counter was sized for (see "Per-unit
+ *                outputs" above)
  * Returns SSA_OK or a negative status.
  */
 int ssa_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch, int total_tokens,
             int max_seqlen, int num_heads, int head_dim, float softmax_scale, float threshold_scale_factor,
-            void* out, int32_t* skip_counter, void* stream);
+            void* out, int32_t* skip_counter, int num_qblocks, void* stream);
 
 /*
  * ssa_fwd plus per-tile diagnostics, for tests. T = ceil(max_seqlen / 128).
@@ -94,7 +109,8 @@ int ssa_fwd(const void* q, const void* k, const void* v, const int32_t* cu_seqle
  */
 int ssa_fwd_ex(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch, int total_tokens,
                int max_seqlen, int num_heads, int head_dim, float softmax_scale, float threshold_scale_factor,
-               void* out, int32_t* skip_counter, uint32_t* decision_bitmap, float* tile_stat, void* stream);
+               void* out, int32_t* skip_counter, int num_qblocks, uint32_t* decision_bitmap, float* tile_stat,
+               void* stream);
 
 /*
  * Calibration pass (commit page, "Triton kernels": full attention that counts
@@ -108,10 +124,25 @@ int ssa_fwd_ex(const void* q, const void* k, const void* v, const int32_t* cu_se
  *                 number of KV tiles j >= 1 with d_j < log2(lambda_k) on the
  *                 dense trajectory. For lambda_k <= 1 this equals ssa_fwd's
  *                 skip count at threshold_scale_factor = lambda_k * S_kv.
+ *   num_qblocks   Q, the count `counts` was sized for
  */
 int ssa_calibrate(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
                   int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
-                  const float* thresholds, int n_thresholds, void* out, int32_t* counts, void* stream);
+                  const float* thresholds, int n_thresholds, void* out, int32_t* counts, int num_qblocks,
+                  void* stream);
+
+/*
+ * ssa_calibrate plus the statistic behind every count, for tests (the
+ * calibration kernel's per-program buffers, commit page "Triton kernels"):
+ *   tile_stat  device float [num_heads][Q][T], T = ceil(max_seqlen / 128), or
+ *              NULL: d_j of every tile on the dense trajectory (+inf for tile
+ *              0; entries past the sequence's last tile are left untouched),
+ *              so that counts[.][.][k] = #{ j : tile_stat[.][.][j] < log2(lambda_k) }.
+ */
+int ssa_calibrate_ex(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                     int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                     const float* thresholds, int n_thresholds, void* out, int32_t* counts, int num_qblocks,
+                     float* tile_stat, void* stream);
 
 /*
  * ssa_fwd_ex with 8-bit Q and K: S = Q K^T runs on E4M3 operands (OCP FP8,
@@ -126,13 +157,14 @@ int ssa_calibrate(const void* q, const void* k, const void* v, const int32_t* cu
  *   q, k        device E4M3 bytes [total_tokens, num_heads, 128] (head_dim must be 128)
  *   v, out      device bf16 [total_tokens, num_heads, 128]
  *   q_descale, k_descale  > 0, finite
- *   skip_counter, decision_bitmap, tile_stat  as in ssa_fwd_ex, each nullable
+ *   skip_counter, num_qblocks, decision_bitmap, tile_stat  as in ssa_fwd_ex
+ *                (the three buffers each nullable)
  * Returns SSA_OK or a negative status (SSA_ERR_UNSUPPORTED for head_dim != 128).
  */
 int ssa_fwd_fp8(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch, int total_tokens,
                 int max_seqlen, int num_heads, int head_dim, float softmax_scale, float q_descale, float k_descale,
-                float threshold_scale_factor, void* out, int32_t* skip_counter, uint32_t* decision_bitmap,
-                float* tile_stat, void* stream);
+                float threshold_scale_factor, void* out, int32_t* skip_counter, int num_qblocks,
+                uint32_t* decision_bitmap, float* tile_stat, void* stream);
 
 /*
  * Per-tensor E4M3 quantisation for ssa_fwd_fp8: y[i] = E4M3(fp32(x[i] * inv_scale)),
@@ -154,7 +186,7 @@ int ssa_quantize_fp8(const void* x, void* y, int64_t n, float inv_scale, void* s
 int ssa_calibrate_fp8(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
                       int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
                       float q_descale, float k_descale, const float* thresholds, int n_thresholds, void* out,
-                      int32_t* counts, void* stream);
+                      int32_t* counts, int num_qblocks, void* stream);
 
 /*
  * threshold_scale_factor = a * exp(b * target_sparsity) (README, "Calibrated
@@ -180,8 +212,10 @@ int ssa_fit_logspace(const double* sparsity, const double* scale_factor, int n, 
  * cu_seqlens; negative status when it is inconsistent. */
 int ssa_num_qblocks(const int32_t* cu_seqlens_host, int batch);
 
-/* Synchronise `stream`, then return and clear this device's kernel status:
- * SSA_OK, SSA_ERR_TIMEOUT, SSA_ERR_DEVICE_ARG or SSA_ERR_CUDA. */
+/* Synchronise `stream`, then return this device's kernel status (SSA_OK,
+ * SSA_ERR_TIMEOUT, SSA_ERR_DEVICE_ARG or SSA_ERR_CUDA) and clear the bits it
+ * read, atomically on the device: an error that a kernel on another stream
+ * records meanwhile is kept for the next call, not lost. */
 int ssa_get_error(void* stream);
 
 /* Static description of a status code. */

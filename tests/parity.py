@@ -9,7 +9,10 @@ and output, fp32 accumulation):
 For lambda <= 1 the running-max trajectory does not depend on decisions, so
 every non-margin tile is compared. For lambda > 1 a margin tile decided the
 other way legitimately changes the rest of the unit's walk; such a unit is
-compared up to that tile and then only checked for finite output.
+compared with the oracle up to that tile, then walked again by the oracle
+with every decision forced to the GPU's (the oracle's replay mode): along
+that trajectory every non-margin decision must be the one the oracle's own
+statistic gives, and the output is held to the same tolerances.
 """
 from __future__ import annotations
 
@@ -63,6 +66,7 @@ class Stats:
         self.tiles = 0
         self.margin_tiles = 0
         self.divergent_units = 0
+        self.replayed_units = 0
 
     def add(self, got, exp):
         d = np.abs(got.astype(np.float64) - exp.astype(np.float64))
@@ -79,10 +83,18 @@ class Stats:
         assert self.mean_abs <= MEAN_ABS, f"{what}: mean abs err {self.mean_abs}"
 
 
-def compare_forward(res, cu, L_seq, out_gpu, skip_gpu, bitmap_gpu, stat_gpu, stats: Stats, what=""):
+def decisions_of(words, nt):
+    """Per-tile decisions (True = skipped) from one unit's bitmap words."""
+    return np.array([(int(words[j >> 5]) >> (j & 31)) & 1 for j in range(nt)], dtype=bool)
+
+
+def compare_forward(res, cu, L_seq, out_gpu, skip_gpu, bitmap_gpu, stat_gpu, stats: Stats, what="", replay=None):
     """Compare oracle result ``res`` (from oracle.walk with per-sequence
     thresholds ``L_seq``) with the GPU's outputs (host arrays: out [total,H,D]
-    fp32, skip [H,Q], bitmap [H,Q,W], stat [H,Q,T])."""
+    fp32, skip [H,Q], bitmap [H,Q,W], stat [H,Q,T]). ``replay(i, forced)``
+    walks unit i again in the oracle with decisions forced ([max_tiles] int8,
+    1 skip / 0 keep / -1 decide); without it a diverged unit is only checked
+    for finite output."""
     units = res["units"]
     gq = global_qblock(cu, units)
     for i, u in enumerate(units):
@@ -92,8 +104,7 @@ def compare_forward(res, cu, L_seq, out_gpu, skip_gpu, bitmap_gpu, stat_gpu, sta
         L = float(L_seq[b])
         d_or = res["dstat"][i, :nt].astype(np.float64)
         dec_or = res["decision"][i, :nt].astype(bool)
-        words = bitmap_gpu[h, gq[i]]
-        dec_gpu = np.array([(int(words[j >> 5]) >> (j & 31)) & 1 for j in range(nt)], dtype=bool)
+        dec_gpu = decisions_of(bitmap_gpu[h, gq[i]], nt)
         margin = np.isfinite(d_or) & (np.abs(d_or - L) <= MARGIN) if math.isfinite(L) else np.zeros(nt, bool)
         stats.tiles += nt
         stats.margin_tiles += int(margin.sum())
@@ -119,14 +130,31 @@ def compare_forward(res, cu, L_seq, out_gpu, skip_gpu, bitmap_gpu, stat_gpu, sta
         got = out_gpu[s0:s0 + n, h]
         if diverged_at < nt:
             stats.divergent_units += 1
-            assert np.all(np.isfinite(got))
+            if replay is None:
+                assert np.all(np.isfinite(got))
+                continue
+            forced = np.full(res["dstat"].shape[1], -1, dtype=np.int8)
+            forced[:nt] = dec_gpu
+            rep = replay(i, forced)
+            d_rep = rep["dstat"][0, :nt].astype(np.float64)
+            free = np.isfinite(d_rep) & (np.abs(d_rep - L) > MARGIN)
+            bad = np.nonzero(free & (dec_gpu != (d_rep < L)))[0]
+            assert bad.size == 0, f"{what}: unit {u}: replayed decisions differ at tiles {bad[:10]}"
+            stats.replayed_units += 1
+            stats.add(got, rep["out"][0, :n])
             continue
         if not margin.any():
             assert int(skip_gpu[h, gq[i]]) == int(res["skips"][i]), f"{what}: unit {u}: skip count"
         stats.add(got, res["out"][i, :n])
 
 
-def compare_calibration(res, cu, cal_L, out_gpu, counts_gpu, stats: Stats, what=""):
+def compare_calibration(res, cu, cal_L, out_gpu, counts_gpu, stats: Stats, what="", stat_gpu=None):
+    """Calibration counts (and output) against the oracle's calibration walk.
+    With the GPU's per-tile statistic ``stat_gpu`` [H,Q,T] (ssa_calibrate_ex)
+    the comparison is tile by tile: each count must equal the number of tiles
+    whose GPU statistic lies below the threshold, and that statistic must give
+    the oracle's decision on every tile more than the margin away from it, so
+    a right count made of two wrong tiles cannot pass."""
     units = res["units"]
     gq = global_qblock(cu, units)
     for i, u in enumerate(units):
@@ -134,11 +162,24 @@ def compare_calibration(res, cu, cal_L, out_gpu, counts_gpu, stats: Stats, what=
         S = int(cu[b + 1] - cu[b])
         nt = (S + TILE - 1) // TILE
         d_or = res["dstat"][i, :nt].astype(np.float64)
+        if stat_gpu is not None:
+            d_gpu = stat_gpu[h, gq[i], :nt].astype(np.float64)
+            fin = np.isfinite(d_or)
+            assert np.all(np.isinf(d_gpu[~fin])), f"{what}: unit {u}: tile-0 statistic not +inf"
+            if fin.any():
+                err = np.abs(d_gpu[fin] - d_or[fin]).max()
+                assert err <= 5e-3, f"{what}: unit {u}: tile statistic differs by {err}"
         for kk, L in enumerate(cal_L):
-            near = int((np.isfinite(d_or) & (np.abs(d_or - L) <= MARGIN)).sum())
+            near_mask = np.isfinite(d_or) & (np.abs(d_or - L) <= MARGIN)
+            near = int(near_mask.sum())
             stats.margin_tiles += near
             diff = abs(int(counts_gpu[h, gq[i], kk]) - int(res["counts"][i, kk]))
             assert diff <= near, f"{what}: unit {u} threshold {kk}: count differs by {diff} ({near} margin tiles)"
+            if stat_gpu is not None:
+                dec_gpu = d_gpu < np.float32(L)
+                assert int(counts_gpu[h, gq[i], kk]) == int(dec_gpu.sum()), f"{what}: unit {u}: count != statistic"
+                bad = np.nonzero(~near_mask & (dec_gpu != (d_or < L)))[0]
+                assert bad.size == 0, f"{what}: unit {u} threshold {kk}: tiles {bad[:10]} decided differently"
         stats.tiles += nt
         s0, n = unit_rows(cu, u)
         stats.add(out_gpu[s0:s0 + n, h], res["out"][i, :n])

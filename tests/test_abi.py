@@ -53,12 +53,12 @@ def test_host_argument_validation(ssa):
     mis = ctypes.c_void_p(0x10008)
     none = None
     args = dict(q=fake, k=fake, v=fake, cu=fake, batch=1, total=256, maxs=256, H=2, D=128, scale=0.0, tsf=0.0,
-                out=fake, sc=None, stream=None)
+                out=fake, sc=None, nq=2, stream=None)
 
     def call(**kw):
         a = dict(args, **kw)
         return L.ssa_fwd(a["q"], a["k"], a["v"], a["cu"], a["batch"], a["total"], a["maxs"], a["H"], a["D"],
-                         a["scale"], a["tsf"], a["out"], a["sc"], a["stream"])
+                         a["scale"], a["tsf"], a["out"], a["sc"], a["nq"], a["stream"])
 
     assert call(q=none) == ssa.SSA_ERR_INVALID_ARG
     assert call(out=none) == ssa.SSA_ERR_INVALID_ARG
@@ -72,17 +72,22 @@ def test_host_argument_validation(ssa):
     assert call(tsf=float("inf")) == ssa.SSA_ERR_INVALID_ARG
     assert call(scale=float("nan")) == ssa.SSA_ERR_INVALID_ARG
     assert call(total=0) == ssa.SSA_OK  # nothing to do, nothing launched
+    assert call(sc=fake, nq=-1) == ssa.SSA_ERR_INVALID_ARG  # a per-unit output needs its q-block count
     th = np.array([1e-3, 0.5], dtype=np.float32)
-    cal = lambda th, n, counts=fake: L.ssa_calibrate(fake, fake, fake, fake, 1, 256, 256, 2, 128, 0.0,
-                                                     th.ctypes.data if th is not None else None, n, fake, counts,
-                                                     None)
+    cal = lambda th, n, counts=fake, nq=2: L.ssa_calibrate(fake, fake, fake, fake, 1, 256, 256, 2, 128, 0.0,
+                                                           th.ctypes.data if th is not None else None, n, fake,
+                                                           counts, nq, None)
     assert cal(th, 0) == ssa.SSA_ERR_INVALID_ARG
     assert cal(th, 33) == ssa.SSA_ERR_INVALID_ARG
     assert cal(None, 2) == ssa.SSA_ERR_INVALID_ARG
     assert cal(th, 2, counts=None) == ssa.SSA_ERR_INVALID_ARG
+    assert cal(th, 2, nq=-1) == ssa.SSA_ERR_INVALID_ARG
     assert cal(np.array([1e-3, 0.0], dtype=np.float32), 2) == ssa.SSA_ERR_INVALID_ARG
-    ex = L.ssa_fwd_ex(fake, fake, fake, fake, 1, 256, 0, 2, 128, 0.0, 10.0, fake, None, fake, None, None)
+    ex = L.ssa_fwd_ex(fake, fake, fake, fake, 1, 256, 0, 2, 128, 0.0, 10.0, fake, None, 2, fake, None, None)
     assert ex == ssa.SSA_ERR_INVALID_ARG  # diagnostics need max_seqlen >= 1
+    cex = L.ssa_calibrate_ex(fake, fake, fake, fake, 1, 256, 0, 2, 128, 0.0, th.ctypes.data, 2, fake, fake, 2,
+                             fake, None)
+    assert cex == ssa.SSA_ERR_INVALID_ARG  # so does the calibration statistic
     assert ssa.lib().ssa_status_string(ssa.SSA_ERR_TIMEOUT)
 
 
@@ -115,7 +120,8 @@ def test_fp8_entry_points_validate_on_the_host(ssa):
     mis = ctypes.c_void_p(0x10008)
 
     def f8(D=128, qd=1.0, kd=1.0, total=256, q=fake, tsf=0.0):
-        return L.ssa_fwd_fp8(q, fake, fake, fake, 1, total, 256, 2, D, 0.0, qd, kd, tsf, fake, None, None, None, None)
+        return L.ssa_fwd_fp8(q, fake, fake, fake, 1, total, 256, 2, D, 0.0, qd, kd, tsf, fake, None, 0, None, None,
+                             None)
 
     assert f8(D=64) == ssa.SSA_ERR_UNSUPPORTED  # E4M3 rows must be 128 bytes
     assert f8(qd=0.0) == ssa.SSA_ERR_INVALID_ARG
@@ -133,6 +139,40 @@ def test_fp8_entry_points_validate_on_the_host(ssa):
     assert qz(mis, fake, 16, 1.0) == ssa.SSA_ERR_UNSUPPORTED
     assert qz(fake, ctypes.c_void_p(0x10004), 16, 1.0) == ssa.SSA_ERR_UNSUPPORTED
     assert qz(fake, fake, 0, 1.0) == ssa.SSA_OK
+
+
+def test_per_unit_outputs_are_checked_before_the_library_is_called(ssa):
+    """Every per-unit output must be [H, Q, inner] with the inner size that
+    max_seqlen (or the threshold count) fixes and one Q shared by all of
+    them; an undersized or misshapen buffer of any of the four kinds is a
+    ValueError before any call. (The exact Q is checked by the kernels
+    against the device copy of cu_seqlens.)"""
+    import torch
+
+    cpu = torch.device("cpu")
+    H, total, batch, max_seqlen = 3, 1000, 2, 700  # T = 6 tiles, 1 bitmap word
+    z = lambda *shape, dt=torch.int32: torch.zeros(shape, dtype=dt)
+    good = ssa._forward_outputs(z(H, 9), z(H, 9, 1), z(H, 9, 6, dt=torch.float32), max_seqlen)
+    assert ssa._per_unit_qblocks(cpu, H, total, batch, good) == 9
+    assert ssa._per_unit_qblocks(cpu, H, total, batch, ssa._forward_outputs(None, None, None, max_seqlen)) == -1
+    bad_forward = [
+        (z(H - 1, 9), None, None),                          # skip_counter: too few heads
+        (z(H, 9, 2), None, None),                           # skip_counter: an inner dimension
+        (None, z(H, 9, 0), None),                           # decision_bitmap: no word per unit
+        (None, z(H, 9), None),                              # decision_bitmap: missing its word axis
+        (None, None, z(H, 9, 5, dt=torch.float32)),         # tile_stat: one tile short
+        (None, None, z(H, 9, 6)),                           # tile_stat: wrong dtype
+        (z(H, 9), z(H, 8, 1), None),                        # two outputs, two q-block counts
+        (z(H, 100), None, None),                            # more q-blocks than 1000 tokens in 2 sequences
+    ]
+    for sc, bm, ts in bad_forward:
+        with pytest.raises((ValueError, TypeError)):
+            ssa._per_unit_qblocks(cpu, H, total, batch, ssa._forward_outputs(sc, bm, ts, max_seqlen))
+    counts = lambda q, n: [(z(H, q, n), "counts", torch.int32, (4,))]
+    assert ssa._per_unit_qblocks(cpu, H, total, batch, counts(9, 4)) == 9
+    for q, n in [(9, 3), (9, 5)]:                           # counts: wrong number of thresholds
+        with pytest.raises(ValueError):
+            ssa._per_unit_qblocks(cpu, H, total, batch, counts(q, n))
 
 
 def test_package_refuses_to_import_without_its_library(tmp_path):

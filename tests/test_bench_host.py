@@ -27,14 +27,14 @@ def test_config_object_is_shared_by_both_arms():
     assert "inputs larger than L2" in cfg["l2"]
 
 
-def _fake_root(tmp_path, traffic_lines, peaks=None):
+def _fake_root(tmp_path, traffic_records, peaks=None):
     src = os.path.join(bench.ROOT, "block_sparse_flashattention_ssa_b200", "csrc")
     dst = tmp_path / "block_sparse_flashattention_ssa_b200" / "csrc"
     dst.mkdir(parents=True)
     for f in ("ssa_kernel.cu", "sm100.cuh"):
         shutil.copy(os.path.join(src, f), dst / f)
     (tmp_path / "profiles").mkdir()
-    (tmp_path / "profiles" / "ssa_attention_wan14b_dram.md").write_text("# x\n" + "\n".join(traffic_lines) + "\n")
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(traffic_records))
     if peaks is not None:
         (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(peaks))
     return str(tmp_path)
@@ -42,19 +42,20 @@ def _fake_root(tmp_path, traffic_lines, peaks=None):
 
 def test_traffic_is_reported_only_for_the_profiled_kernel_source(tmp_path, monkeypatch):
     h = bench.kernel_source_hash()
-    root = _fake_root(tmp_path, [f"traffic: hash={h} workload=wan14b tsf=24285.8487367675 bytes=3567250000",
-                                 f"traffic: hash={h} workload=wan14b tsf=0 bytes=3591750000",
-                                 "traffic: hash=0000000000000000 workload=wan14b tsf=5000 bytes=1"])
+    root = _fake_root(tmp_path, [{"hash": h, "workload": "wan14b", "tsf": 24285.8487367675, "bytes": 3567250000},
+                                 {"hash": h, "workload": "wan14b", "tsf": 0.0, "bytes": 3591750000},
+                                 {"hash": "0000000000000000", "workload": "wan14b", "tsf": 5000.0, "bytes": 1}])
     monkeypatch.setattr(bench, "ROOT", root)
+    path = os.path.join(root, "profiles", "traffic.json")
     assert bench.kernel_source_hash() == h
-    assert bench.measured_traffic("wan14b", 24285.8487367675) == 3567250000.0
-    assert bench.measured_traffic("wan14b", 0.0) == 3591750000.0
-    assert bench.measured_traffic("wan14b", 5000.0) is None  # another kernel source
-    assert bench.measured_traffic("wan5b", 0.0) is None
+    assert bench.measured_traffic("wan14b", 24285.8487367675, path) == 3567250000.0
+    assert bench.measured_traffic("wan14b", 0.0, path) == 3591750000.0
+    assert bench.measured_traffic("wan14b", 5000.0, path) is None  # another kernel source
+    assert bench.measured_traffic("wan5b", 0.0, path) is None
     # any edit of the kernel sources invalidates the stored counters
     with open(os.path.join(root, "block_sparse_flashattention_ssa_b200", "csrc", "sm100.cuh"), "a") as f:
         f.write("\n// edited\n")
-    assert bench.measured_traffic("wan14b", 0.0) is None
+    assert bench.measured_traffic("wan14b", 0.0, path) is None
 
 
 def test_peaks_prefer_the_measured_file(tmp_path, monkeypatch):

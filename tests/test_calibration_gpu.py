@@ -68,3 +68,41 @@ def test_forward_at_a_trial_threshold_matches_the_calibration_count(ssa):
     for i, lam in enumerate(trials):
         _, skip = _skip_ratio(ssa, dq, dk, dv, dcu, w, lam * S)
         assert np.array_equal(skip.cpu().numpy(), counts[:, :, i].cpu().numpy()), lam
+
+
+def test_head_sharded_calibration_equals_the_unsharded_one(ssa):
+    """Heads split over two ranks (contiguous head slices, each copied into
+    its own [T, H/2, D] tensors as a rank would hold them): each shard counts
+    with ssa_calibrate, the per-sequence count sums are added (the all-reduce
+    of a head-sharded run, here the other shard's sums added in place of the
+    collective) and every shard fits. Counts, sums and (a, b) must equal the
+    single-call calibration over all heads bit for bit."""
+    from block_sparse_flashattention_ssa_b200 import calibration as cal
+
+    w = synth.VARLEN
+    q, k, v = synth.generate(w)
+    cu = w.cu_seqlens
+    dq, dk, dv, dcu = parity.to_device(q, k, v, cu)
+    trials = cal.DEFAULT_TRIALS
+    _, counts_all = ssa.calibrate(dq, dk, dv, dcu, w.max_seqlen, list(trials))
+    ssa.check_device()
+    whole = cal.calibrate(dq, dk, dv, dcu, w.max_seqlen, trials)
+    ssa.check_device()
+    world = 2
+    shards = [cal.shard_heads(w.H, world, r) for r in range(world)]
+    per_rank, seq_sums = [], []
+    for hr in shards:
+        sl = slice(hr.start, hr.stop)
+        sq, sk, sv = (t[:, sl].contiguous() for t in (dq, dk, dv))
+        _, c = ssa.calibrate(sq, sk, sv, dcu, w.max_seqlen, list(trials))
+        ssa.check_device()
+        assert torch.equal(c, counts_all[sl]), hr  # a head's counts do not depend on the other heads
+        per_rank.append((sq, sk, sv))
+        seq_sums.append(cal.sequence_counts(c.cpu().numpy(), cu))
+    assert np.array_equal(seq_sums[0] + seq_sums[1], cal.sequence_counts(counts_all.cpu().numpy(), cu))
+    for r, (sq, sk, sv) in enumerate(per_rank):
+        other = seq_sums[1 - r]
+        got = cal.calibrate(sq, sk, sv, dcu, w.max_seqlen, trials, total_heads=w.H, allreduce=lambda s: s + other)
+        ssa.check_device()
+        assert (got.a, got.b, got.s_min, got.s_max) == (whole.a, whole.b, whole.s_min, whole.s_max), r
+        assert got.points == whole.points

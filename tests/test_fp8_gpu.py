@@ -49,30 +49,15 @@ class Fp8Case(Case):
         torch.cuda.synchronize()
         assert np.array_equal(self.dq8.cpu().numpy(), self.q8) and np.array_equal(self.dk8.cpu().numpy(), self.k8)
         # oracle softmax scale: 1/sqrt(D) * q_descale * k_descale, in the order the library forms it
-        self.scale = 1.0 / math.sqrt(w.D) * (float(self.q_ds) * float(self.k_ds))
+        self.oracle_scale = 1.0 / math.sqrt(w.D) * (float(self.q_ds) * float(self.k_ds))
 
-    def fwd(self, tsf, ex=True):
-        H = self.w.H
-        skip = torch.full((H, self.Q), -1, dtype=torch.int32, device="cuda")
-        bitmap = torch.zeros((H, self.Q, self.ssa.bitmap_words(self.w.max_seqlen)), dtype=torch.int32, device="cuda")
-        stat = torch.full((H, self.Q, self.T), float("nan"), dtype=torch.float32, device="cuda")
-        out = torch.full_like(self.dv, float("nan"))
+    def call(self, tsf, out, skip, bitmap, stat):
         self.ssa.fwd_fp8(self.dq8, self.dk8, self.dv, self.dcu, self.w.max_seqlen, float(self.q_ds),
-                         float(self.k_ds), tsf, out=out, skip_counter=skip, decision_bitmap=bitmap if ex else None,
-                         tile_stat=stat if ex else None)
-        self.ssa.check_device()
-        return (parity.bf16_host(out), skip.cpu().numpy(), bitmap.cpu().numpy().view(np.uint32),
-                stat.cpu().numpy())
+                         float(self.k_ds), tsf, out=out, skip_counter=skip, decision_bitmap=bitmap, tile_stat=stat)
 
 
 def _check(case, tsf, units=None, what=""):
-    out, skip, bitmap, stat = case.fwd(tsf)
-    res = oracle.walk(case.q, case.k, case.v, case.cu, case.w.H, case.w.D, softmax_scale=case.scale, tsf=tsf,
-                      units=units, max_tiles=case.T)
-    st = parity.Stats()
-    parity.compare_forward(res, case.cu, case.L_seq(tsf), out, skip, bitmap, stat, st, what=f"{what} tsf={tsf}")
-    st.check(f"{what} tsf={tsf}")
-    return st, skip
+    return check_forward(case, tsf, units=units, what=what, plain=True)
 
 
 def test_quantiser_matches_the_format_definition_bit_for_bit(ssa):
@@ -121,8 +106,7 @@ def test_fp8_calibration_counts_and_forward_equivalence(ssa):
     out, counts = ssa.calibrate_fp8(case.dq8, case.dk8, case.dv, case.dcu, w.max_seqlen, float(case.q_ds),
                                     float(case.k_ds), lams)
     ssa.check_device()
-    res = oracle.walk(case.q, case.k, case.v, case.cu, w.H, w.D, softmax_scale=case.scale, cal_lambdas=lams,
-                      max_tiles=case.T)
+    res = case.walk(cal_lambdas=lams)
     st = parity.Stats()
     parity.compare_calibration(res, case.cu, [oracle.lambda_log2(x) for x in lams], parity.bf16_host(out),
                                counts.cpu().numpy(), st, what="calib fp8")
@@ -138,3 +122,24 @@ def test_fp8_calibration_counts_and_forward_equivalence(ssa):
     for kk, lam in enumerate(lams):
         _, skip, _, _ = one.fwd(lam * 1024)
         assert np.array_equal(skip, c1[:, :, kk]), lam
+
+
+def test_fp8_wan14b_at_the_benchmarked_threshold(ssa):
+    """The benchmark's E4M3 row: S = 75,600, H = 40, D = 128 at the threshold
+    it uses for target 0.7 (resolved from the bf16 calibration and fit on the
+    same input) and dense, 12 sampled units; the call without diagnostics
+    equals the diagnostic one bit for bit."""
+    from block_sparse_flashattention_ssa_b200 import calibration as cal
+
+    w = synth.WAN14B
+    bf = Case(ssa, w)
+    c = cal.calibrate(bf.dq, bf.dk, bf.dv, bf.dcu, w.max_seqlen)
+    ssa.check_device()
+    tsf = ssa.resolve(c.a, c.b, 0.7)
+    del bf
+    torch.cuda.empty_cache()
+    case = Fp8Case(ssa, w)
+    units = oracle.sample_units(case.cu, w.H, 12, seed=22)
+    _check(case, 0.0, units=units, what="wan14b fp8 dense")
+    _, skip = _check(case, tsf, units=units, what="wan14b fp8 target 0.7")
+    assert skip.sum() > 0

@@ -8,6 +8,8 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
 
 def _free_port():
     with socket.socket() as s:
@@ -55,3 +57,32 @@ def test_single_rank_is_identity():
 
     assert bench.max_over_ranks(12.5, 1) == 12.5
     assert bench.weak_scaling_value(4e12, 1, 1000.0) == pytest.approx(4.0)
+
+
+def test_bench_gpus_flag_launches_that_many_ranks():
+    """`python bench.py --gpus 2` re-executes itself under
+    torch.distributed.run with two local ranks (127.0.0.1); rank 0 alone
+    prints the line of the reference arm (here on the tiny workload, CPU
+    only) with n_gpus = 2, the other rank exits 0 without work."""
+    import json
+    import subprocess
+    import sys
+
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "0", "--cpu-seconds", "0.5"],
+                       capture_output=True, text=True, timeout=240, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    assert lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
+
+
+def test_bench_refuses_a_world_size_other_than_gpus():
+    import subprocess
+    import sys
+
+    env = dict(os.environ, WORLD_SIZE="3", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1"], capture_output=True, text=True, timeout=120,
+                       env=env, cwd=ROOT)
+    assert r.returncode == 2 and "WORLD_SIZE=3" in r.stderr

@@ -270,6 +270,28 @@ def test_threshold_conversion_page_pin():
     assert oracle.score_scale(0.0, 128) == pytest.approx(1 / math.sqrt(128) / math.log(2), rel=1e-7)
 
 
+def test_raw_lambda_conversion_pins():
+    """The calibration trials are raw lambda values compared as log2(lambda):
+    the page constant (lambda 0.61557 replacing log2-space -0.7) holds for the
+    raw conversion too; exact powers of two map to their exponents (a natural
+    log or a missing fp32 rounding would not); 2**L gives lambda back to fp32
+    precision for every printed trial; and the raw conversion agrees with the
+    scale-factor one, lambda = tsf / S_kv, where tsf / S_kv is exact."""
+    (lam, raw), = first("page_constants.txt", "lambda_log2")
+    assert oracle.lambda_log2(lam) == pytest.approx(raw, abs=1e-4)
+    for e in range(-24, 4):
+        assert oracle.lambda_log2(2.0 ** e) == float(e)
+    (trials,) = first("page_constants.txt", "trials")
+    for x in trials:
+        L = oracle.lambda_log2(x)
+        assert np.float32(L) == L  # an fp32 value
+        assert 2.0 ** L == pytest.approx(x, rel=3e-7 * max(1.0, abs(L)))
+        for S in [1024, 65536]:  # powers of two: x * S / S is exact in double
+            assert oracle.lambda_log2(x) == oracle.threshold_log2(x * S, S)
+    assert oracle.lambda_log2(0.0) == -math.inf and oracle.lambda_log2(-1.0) == -math.inf
+    assert oracle.lambda_log2(1.0) == 0.0
+
+
 # ------------------------------------------------------------ fit / resolve
 
 

@@ -33,6 +33,8 @@ def ssa():
 class Case:
     """Host inputs, their device copies and the GPU runs of one workload."""
 
+    oracle_scale = 0.0  # softmax_scale the oracle is given (0: 1/sqrt(D))
+
     def __init__(self, ssa, w: synth.Workload, q=None, k=None, v=None):
         self.ssa, self.w = ssa, w
         if q is None:
@@ -43,29 +45,49 @@ class Case:
         self.Q = ssa.num_qblocks(self.cu)
         self.T = ssa.max_tiles(w.max_seqlen)
 
+    def call(self, tsf, out, skip, bitmap, stat):
+        self.ssa.fwd(self.dq, self.dk, self.dv, self.dcu, self.w.max_seqlen, tsf, out=out, skip_counter=skip,
+                     decision_bitmap=bitmap, tile_stat=stat)
+
     def fwd(self, tsf, ex=True):
+        """One forward; ex=False runs the call without diagnostics (the
+        kernels the benchmark times)."""
         H = self.w.H
         skip = torch.full((H, self.Q), -1, dtype=torch.int32, device="cuda")
         bitmap = torch.zeros((H, self.Q, self.ssa.bitmap_words(self.w.max_seqlen)), dtype=torch.int32, device="cuda")
         stat = torch.full((H, self.Q, self.T), float("nan"), dtype=torch.float32, device="cuda")
-        out = torch.full_like(self.dq, float("nan"))
-        self.ssa.fwd(self.dq, self.dk, self.dv, self.dcu, self.w.max_seqlen, tsf, out=out, skip_counter=skip,
-                     decision_bitmap=bitmap if ex else None, tile_stat=stat if ex else None)
+        out = torch.full_like(self.dv, float("nan"))
+        self.call(tsf, out, skip, bitmap if ex else None, stat if ex else None)
         self.ssa.check_device()
         return (parity.bf16_host(out), skip.cpu().numpy(), bitmap.cpu().numpy().view(np.uint32),
                 stat.cpu().numpy())
+
+    def walk(self, **kw):
+        return oracle.walk(self.q, self.k, self.v, self.cu, self.w.H, self.w.D, softmax_scale=self.oracle_scale,
+                           max_tiles=self.T, **kw)
 
     def L_seq(self, tsf):
         return [oracle.threshold_log2(tsf, s) for s in self.w.seqlens]
 
 
-def check_forward(case, tsf, units=None, what=""):
+def check_forward(case, tsf, units=None, what="", plain=False):
+    """The diagnostic forward against the oracle (decisions, statistics,
+    skip counts, outputs; diverged units replayed). With ``plain`` the call
+    without diagnostics runs too and must give the same output bit for bit
+    and the same skip counts, so the benchmarked kernels are held to the
+    same check."""
     out, skip, bitmap, stat = case.fwd(tsf)
-    res = oracle.walk(case.q, case.k, case.v, case.cu, case.w.H, case.w.D, tsf=tsf, units=units, max_tiles=case.T)
+    if plain:
+        out_p, skip_p, _, _ = case.fwd(tsf, ex=False)
+        np.testing.assert_array_equal(out_p.view(np.uint32), out.view(np.uint32), err_msg=f"{what} tsf={tsf}")
+        np.testing.assert_array_equal(skip_p, skip, err_msg=f"{what} tsf={tsf}")
+    res = case.walk(tsf=tsf, units=units)
+    replay = lambda i, forced: case.walk(tsf=tsf, units=res["units"][i:i + 1], forced=forced[None, :])
     st = parity.Stats()
-    parity.compare_forward(res, case.cu, case.L_seq(tsf), out, skip, bitmap, stat, st, what=f"{what} tsf={tsf}")
+    parity.compare_forward(res, case.cu, case.L_seq(tsf), out, skip, bitmap, stat, st, what=f"{what} tsf={tsf}",
+                           replay=replay)
     st.check(f"{what} tsf={tsf}")
-    assert st.divergent_units <= max(1, len(res["units"]) // 50), st.divergent_units
+    assert st.divergent_units <= max(1, len(res["units"]) // 10), st.divergent_units
     return st, skip
 
 
@@ -74,7 +96,7 @@ def test_tiny_full(ssa):
     case = Case(ssa, synth.TINY)
     ratios = []
     for tsf in synth.TINY.tsf:
-        st, skip = check_forward(case, tsf, what="tiny")
+        st, skip = check_forward(case, tsf, what="tiny", plain=True)
         ratios.append(skip.sum() / st.tiles)
     assert ratios[0] == 0 and ratios[2] >= ratios[1]
 
@@ -90,7 +112,7 @@ def test_ragged_varlen(ssa, D):
     cu = w.cu_seqlens
     case = Case(ssa, w, q, k, v)
     for tsf in [0.0, 50.0, 300.0, 2000.0]:
-        check_forward(case, tsf, what=f"ragged D={D}")
+        check_forward(case, tsf, what=f"ragged D={D}", plain=True)
 
 
 def test_skip_path_without_skips_is_bitwise_dense(ssa):
@@ -109,7 +131,7 @@ def test_wan5b_threshold_sweep(ssa):
     case = Case(ssa, synth.WAN5B)
     units = oracle.sample_units(case.cu, case.w.H, 32, seed=1)
     for tsf in synth.WAN5B.tsf:
-        check_forward(case, tsf, units=units, what="wan5b")
+        check_forward(case, tsf, units=units, what="wan5b", plain=True)
 
 
 def test_wan14b_resolved_thresholds(ssa):
@@ -119,7 +141,28 @@ def test_wan14b_resolved_thresholds(ssa):
     units = oracle.sample_units(case.cu, case.w.H, 12, seed=2)
     a, b = synth.EXAMPLE_FORMULA
     for tsf in [0.0] + [ssa.resolve(a, b, s) for s in synth.TARGET_SPARSITIES]:
-        check_forward(case, tsf, units=units, what="wan14b")
+        check_forward(case, tsf, units=units, what="wan14b", plain=True)
+
+
+def test_wan14b_at_the_benchmarked_thresholds(ssa):
+    """The benchmark's own step: S = 75,600, H = 40, D = 128 at the
+    thresholds it resolves (ssa_calibrate on this input, one fit point per
+    trial, the log-space fit, a*exp(b*s) at s = 0.5, 0.7, 0.9; lambda reaches
+    about 5 at 0.9) and dense. The call without diagnostics (the timed
+    kernels) must equal the diagnostic call bit for bit, which is compared
+    with the oracle on 16 sampled units; skip ratios land near the targets."""
+    from block_sparse_flashattention_ssa_b200 import calibration as cal
+
+    case = Case(ssa, synth.WAN14B)
+    c = cal.calibrate(case.dq, case.dk, case.dv, case.dcu, case.w.max_seqlen)
+    ssa.check_device()
+    units = oracle.sample_units(case.cu, case.w.H, 16, seed=21)
+    tiles = case.w.H * case.T * case.T
+    check_forward(case, 0.0, units=units, what="wan14b bench dense", plain=True)
+    for target in synth.TARGET_SPARSITIES:
+        tsf = ssa.resolve(c.a, c.b, target)
+        st, skip = check_forward(case, tsf, units=units, what=f"wan14b bench target {target}", plain=True)
+        assert abs(skip.sum() / tiles - target) < 0.15, (target, tsf, skip.sum() / tiles)
 
 
 def test_varlen_batch(ssa):
@@ -127,18 +170,25 @@ def test_varlen_batch(ssa):
     tsf = 5000 with lambda per sequence, 16 sampled units."""
     case = Case(ssa, synth.VARLEN)
     units = oracle.sample_units(case.cu, case.w.H, 16, seed=3)
-    check_forward(case, 5000.0, units=units, what="varlen")
+    check_forward(case, 5000.0, units=units, what="varlen", plain=True)
 
 
 def check_calibration(case, units=None, what=""):
+    """ssa_calibrate_ex (counts and every tile's statistic) against the
+    oracle's calibration walk, tile by tile; plain ssa_calibrate must give
+    the same output and counts bit for bit."""
     lams = synth.CALIB_THRESHOLDS
-    out, counts = case.ssa.calibrate(case.dq, case.dk, case.dv, case.dcu, case.w.max_seqlen, lams)
+    stat = torch.full((case.w.H, case.Q, case.T), float("nan"), dtype=torch.float32, device="cuda")
+    out, counts = case.ssa.calibrate(case.dq, case.dk, case.dv, case.dcu, case.w.max_seqlen, lams, tile_stat=stat)
     case.ssa.check_device()
-    res = oracle.walk(case.q, case.k, case.v, case.cu, case.w.H, case.w.D, cal_lambdas=lams, units=units,
-                      max_tiles=case.T)
+    out_p, counts_p = case.ssa.calibrate(case.dq, case.dk, case.dv, case.dcu, case.w.max_seqlen, lams)
+    case.ssa.check_device()
+    assert torch.equal(out.view(torch.int16), out_p.view(torch.int16)) and torch.equal(counts, counts_p)
+    res = case.walk(cal_lambdas=lams, units=units)
     st = parity.Stats()
     cal_L = [oracle.lambda_log2(x) for x in lams]
-    parity.compare_calibration(res, case.cu, cal_L, parity.bf16_host(out), counts.cpu().numpy(), st, what=what)
+    parity.compare_calibration(res, case.cu, cal_L, parity.bf16_host(out), counts.cpu().numpy(), st, what=what,
+                               stat_gpu=stat.cpu().numpy())
     st.check(what)
     return counts.cpu().numpy()
 
@@ -229,11 +279,43 @@ def test_host_memory_is_refused_before_any_launch(ssa):
     host_skip = torch.full((2, 2), -1, dtype=torch.int32).pin_memory()
     stream = vp(torch.cuda.current_stream().cuda_stream)
     rc = L.ssa_fwd(vp(case.dq.data_ptr()), vp(case.dk.data_ptr()), vp(case.dv.data_ptr()), vp(host_cu.data_ptr()),
-                   1, 200, 200, 2, 64, 0.0, 10.0, vp(out.data_ptr()), None, stream)
+                   1, 200, 200, 2, 64, 0.0, 10.0, vp(out.data_ptr()), None, 0, stream)
     assert rc == ssa.SSA_ERR_INVALID_ARG
     rc = L.ssa_fwd(vp(case.dq.data_ptr()), vp(case.dk.data_ptr()), vp(case.dv.data_ptr()), vp(case.dcu.data_ptr()),
-                   1, 200, 200, 2, 64, 0.0, 10.0, vp(out.data_ptr()), vp(host_skip.data_ptr()), stream)
+                   1, 200, 200, 2, 64, 0.0, 10.0, vp(out.data_ptr()), vp(host_skip.data_ptr()), 2, stream)
     assert rc == ssa.SSA_ERR_INVALID_ARG
     torch.cuda.synchronize()
     assert ssa.get_error() == ssa.SSA_OK
     assert bool((out == 7.0).all()) and bool((host_skip == -1).all())  # nothing ran
+
+
+def test_per_unit_outputs_sized_for_another_batch_are_never_written(ssa):
+    """Per-unit outputs whose q-block count differs from the one cu_seqlens
+    gives (too few or too many rows, or a sequence longer than max_seqlen for
+    the diagnostics) make every kernel write nothing and report
+    SSA_ERR_DEVICE_ARG; the right count works on the same buffers' sizes."""
+    w = synth.Workload("two", [(1, 1, 300), (1, 1, 700)], H=2, D=64, seed=0)  # Q = 3 + 6
+    case = Case(ssa, w)
+    assert case.Q == 9
+    lams = [1e-3, 0.5]
+    for q_rows in (case.Q - 1, case.Q + 1):
+        out = torch.full_like(case.dq, 7.0)
+        skip = torch.full((w.H, q_rows), -1, dtype=torch.int32, device="cuda")
+        ssa.fwd(case.dq, case.dk, case.dv, case.dcu, w.max_seqlen, 10.0, out=out, skip_counter=skip)
+        assert ssa.get_error() == ssa.SSA_ERR_DEVICE_ARG
+        counts = torch.full((w.H, q_rows, 2), -1, dtype=torch.int32, device="cuda")
+        ssa.calibrate(case.dq, case.dk, case.dv, case.dcu, w.max_seqlen, lams, out=out, counts=counts)
+        assert ssa.get_error() == ssa.SSA_ERR_DEVICE_ARG
+        assert bool((out == 7.0).all()) and bool((skip == -1).all()) and bool((counts == -1).all())
+    # diagnostics sized for a shorter max_seqlen than the batch holds
+    short = 300
+    bitmap = torch.zeros((w.H, case.Q, ssa.bitmap_words(short)), dtype=torch.int32, device="cuda")
+    stat = torch.full((w.H, case.Q, ssa.max_tiles(short)), -1.0, dtype=torch.float32, device="cuda")
+    out = torch.full_like(case.dq, 7.0)
+    ssa.fwd(case.dq, case.dk, case.dv, case.dcu, short, 10.0, out=out, decision_bitmap=bitmap, tile_stat=stat)
+    assert ssa.get_error() == ssa.SSA_ERR_DEVICE_ARG
+    assert bool((out == 7.0).all()) and bool((bitmap == 0).all()) and bool((stat == -1.0).all())
+    # the right count: written, no error
+    skip = torch.full((w.H, case.Q), -1, dtype=torch.int32, device="cuda")
+    ssa.fwd(case.dq, case.dk, case.dv, case.dcu, w.max_seqlen, 10.0, out=out, skip_counter=skip)
+    assert ssa.get_error() == ssa.SSA_OK and bool((skip >= 0).all())
