@@ -49,7 +49,9 @@ def _load():
         L.oracle_fit_logspace.argtypes = [vp, vp, i32, vp, vp, vp, vp]
         L.oracle_walk.restype = i32
         L.oracle_walk.argtypes = [vp, vp, vp, vp, i32, i32, i32, f64, i32, vp, vp, i32, i32, vp, i32, vp,
-                                  vp, vp, vp, vp, vp, i32]
+                                  vp, vp, vp, vp, vp, i32, f64, f64, f64, i32]
+        L.oracle_e4m3_nearest.restype = f64
+        L.oracle_e4m3_nearest.argtypes = [f64]
         _lib = L
     return _lib
 
@@ -120,13 +122,26 @@ def sample_units(cu_seqlens, H, n, seed=0):
     return np.asarray(chosen, dtype=np.int32).reshape(-1, 3)
 
 
+def e4m3_nearest(x: float) -> float:
+    """Nearest E4M3 value of x >= 0 (ties to even, saturating at 448)."""
+    return float(_load().oracle_e4m3_nearest(float(x)))
+
+
+P_SHIFT = 8.0  # sigma of the 8-bit P.V reading: P = 2^(s2 - r + sigma) <= 256
+P_LAG = 0.0    # tau: the integer reference r follows ceil(m) as soon as m exceeds it
+
+
 def walk(q, k, v, cu_seqlens, H, D, *, softmax_scale=0.0, units=None, tsf=None, L_seq=None,
-         cal_lambdas=None, forced=None, max_tiles=None, nthreads=None):
+         cal_lambdas=None, forced=None, max_tiles=None, nthreads=None, p_e4m3=False, p_shift=P_SHIFT,
+         p_lag=P_LAG, out_scale=1.0):
     """Run the tiled skip-softmax walk on CPU.
 
     q, k, v: uint16 bf16 patterns [total_tokens, H, D]. Either ``tsf`` (one
     threshold_scale_factor for every sequence), ``L_seq`` (per-sequence log2
     thresholds) or ``cal_lambdas`` (calibration mode: raw lambda trials).
+    ``p_e4m3`` selects the 8-bit P.V reading (P rounded to E4M3 against a
+    per-row integer reference, see oracle.cpp); ``out_scale`` multiplies
+    the outputs (the V descale when v holds decoded E4M3 values).
     Returns a dict with ``out`` [n_units, 128, D] fp32, ``dstat`` and
     ``decision`` [n_units, max_tiles], ``skips`` [n_units] and, in calibration
     mode, ``counts`` [n_units, n_cal].
@@ -164,7 +179,8 @@ def walk(q, k, v, cu_seqlens, H, D, *, softmax_scale=0.0, units=None, tsf=None, 
                        float(softmax_scale), mode, ptr(L_seq) if mode == 0 else None,
                        ptr(L_cal) if mode == 1 else None, n_cal, n, units.ctypes.data, max_tiles,
                        ptr(forced), out.ctypes.data, dstat.ctypes.data, decision.ctypes.data, skips.ctypes.data,
-                       counts.ctypes.data if mode == 1 else None, nthreads or min(64, os.cpu_count() or 1))
+                       counts.ctypes.data if mode == 1 else None, 1 if p_e4m3 else 0, float(p_shift),
+                       float(p_lag), float(out_scale), nthreads or min(64, os.cpu_count() or 1))
     if rc != 0:
         raise ValueError("oracle_walk: bad arguments")
     res = dict(out=out, dstat=dstat, decision=decision, skips=skips, units=units, max_tiles=max_tiles)

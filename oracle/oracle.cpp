@@ -27,6 +27,15 @@
 //  * rows past the sequence end do not vote, columns past it are -inf;
 //  * no clamp of lambda to 1;
 //  * probabilities and accumulators in double.
+// The 8-bit P.V reading (the variant with E4M3 Q, K and V): V arrives decoded
+// (each E4M3 value is exact in bf16) and its per-tensor scale multiplies the
+// output; each kept tile's probabilities are taken against a per-row integer
+// reference exponent r and shifted by sigma, P = 2^(s2 - r + sigma), and the
+// P.V product uses P rounded to the nearest E4M3 value (ties to even,
+// saturating at 448) while the row sum l adds the unrounded P. r starts at
+// ceil of the first kept tile's max and moves to ceil(m) whenever the
+// running max m rises above r + tau, rescaling O and l by 2^(r_old - r_new)
+// (a power of two). With tau = 0 and sigma = 8 every P lies in (0, 256].
 // Parity pins for every function live in tests/test_oracle.py.
 #include <algorithm>
 #include <atomic>
@@ -54,7 +63,27 @@ struct Problem {
   const int32_t* cu;
   int batch, H, D;
   float c;  // fp32(softmax_scale * log2 e)
+  int p_e4m3;        // 1: the 8-bit P.V reading above
+  double p_shift;    // sigma
+  double p_lag;      // tau
+  double out_scale;  // multiplies O / l (the V descale)
 };
+
+// Nearest E4M3 value of x >= 0 (OCP 8-bit floating point without infinities:
+// 4 exponent bits with bias 7 and 3 mantissa bits, so a binade 2^e holds 8
+// values 2^(e-3) apart, e >= -6, the subnormals continuing the spacing 2^-9
+// down to 0; the largest finite value is 448). Ties go to the even multiple of
+// the spacing; values from 448 up saturate to 448.
+double e4m3_nearest(double x) {
+  if (!(x > 0.0)) return 0.0;
+  if (x >= 448.0) return 448.0;
+  int e2;
+  std::frexp(x, &e2);  // x = f * 2^e2 with f in [0.5, 1): the binade is 2^(e2 - 1)
+  const int e = std::max(e2 - 1, -6);
+  const double spacing = std::ldexp(1.0, e - 3);
+  const double q = std::nearbyint(x / spacing);  // round half to even (default rounding mode)
+  return std::min(q * spacing, 448.0);
+}
 
 struct UnitResult {
   float* out;        // [128][D]
@@ -82,6 +111,7 @@ void walk_unit(const Problem& P, int seq, int head, int qb, int mode, float L, c
 
   std::vector<float> m(nrows, -inf);
   std::vector<double> l(nrows, 0.0), O(static_cast<size_t>(nrows) * D, 0.0);
+  std::vector<double> ref(nrows, -std::numeric_limits<double>::infinity());  // integer reference (8-bit P)
   std::vector<float> s2(static_cast<size_t>(nrows) * kTile);
   std::vector<double> kcol(D), vrow(D);
   int skips = 0;
@@ -127,16 +157,26 @@ void walk_unit(const Problem& P, int seq, int head, int qb, int mode, float L, c
     // Online softmax update with this tile.
     for (int r = 0; r < nrows; ++r) {
       const float mn = std::max(m[r], tmax[r]);
-      const double alpha = std::exp2(static_cast<double>(m[r]) - static_cast<double>(mn));  // 0 when m = -inf
-      double rowsum = 0.0;
       double* orow = &O[static_cast<size_t>(r) * D];
+      // reference the probabilities are taken against, and the O/l rescale
+      double refp = mn, alpha = std::exp2(static_cast<double>(m[r]) - static_cast<double>(mn));  // 0 when m = -inf
+      if (P.p_e4m3) {
+        alpha = 1.0;
+        if (std::isinf(ref[r]) || static_cast<double>(mn) > ref[r] + P.p_lag) {
+          const double nr = std::ceil(static_cast<double>(mn));
+          alpha = std::isinf(ref[r]) ? 0.0 : std::exp2(ref[r] - nr);
+          ref[r] = nr;
+        }
+        refp = ref[r] - P.p_shift;
+      }
+      double rowsum = 0.0;
       for (int d = 0; d < D; ++d) orow[d] *= alpha;
       for (int c = c0; c < c1; ++c) {
-        const double p = std::exp2(static_cast<double>(s2[static_cast<size_t>(r) * kTile + (c - c0)]) -
-                                   static_cast<double>(mn));
+        const double p = std::exp2(static_cast<double>(s2[static_cast<size_t>(r) * kTile + (c - c0)]) - refp);
         rowsum += p;
+        const double pv = P.p_e4m3 ? e4m3_nearest(p) : p;  // the factor the P.V product uses
         const uint16_t* vr = &P.v[((base + c) * H + head) * D];
-        for (int d = 0; d < D; ++d) orow[d] += p * bf16_to_double(vr[d]);
+        for (int d = 0; d < D; ++d) orow[d] += pv * bf16_to_double(vr[d]);
       }
       l[r] = l[r] * alpha + rowsum;
       m[r] = mn;
@@ -149,7 +189,7 @@ void walk_unit(const Problem& P, int seq, int head, int qb, int mode, float L, c
   for (int r = 0; r < kTile; ++r)
     for (int d = 0; d < D; ++d)
       R.out[static_cast<size_t>(r) * D + d] =
-          r < nrows ? static_cast<float>(O[static_cast<size_t>(r) * D + d] / l[r]) : 0.0f;
+          r < nrows ? static_cast<float>(O[static_cast<size_t>(r) * D + d] / l[r] * P.out_scale) : 0.0f;
   if (R.skips) *R.skips = skips;
   if (R.counts)
     for (int kk = 0; kk < n_cal; ++kk) R.counts[kk] = counts[kk];
@@ -217,18 +257,25 @@ int oracle_fit_logspace(const double* s, const double* sf, int n, double* a, dou
   return 0;
 }
 
+// Nearest E4M3 value (exported for its pins).
+double oracle_e4m3_nearest(double x) { return e4m3_nearest(x); }
+
 // Walk a list of (sequence, head, query-block) units.
 //   mode 0: forward with skipping; L_seq[b] is sequence b's threshold.
 //   mode 1: calibration; never skips, counts d < L_cal[k] for each k.
 // forced (nullable, [n_units][max_tiles]): -1 decide, 0 keep, 1 skip (mode 0).
 // Outputs per unit: out [128][D] fp32 (rows past the end are 0), dstat
 // [max_tiles] (+inf at tile 0, NaN past the end), decision [max_tiles],
-// skips, counts [n_cal]. Returns 0, or -1 on a bad argument.
+// skips, counts [n_cal]. p_e4m3 selects the 8-bit P.V reading (p_shift =
+// sigma, p_lag = tau); out_scale multiplies every output (1 for bf16 V).
+// Returns 0, or -1 on a bad argument.
 int oracle_walk(const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* cu_seqlens, int batch,
                 int H, int D, double softmax_scale, int mode, const float* L_seq, const float* L_cal, int n_cal,
                 int n_units, const int32_t* units, int max_tiles, const int8_t* forced, float* out, float* dstat,
-                uint8_t* decision, int32_t* skips, int32_t* cal_counts, int nthreads) {
+                uint8_t* decision, int32_t* skips, int32_t* cal_counts, int p_e4m3, double p_shift, double p_lag,
+                double out_scale, int nthreads) {
   if (!q || !k || !v || !cu_seqlens || !units || !out || batch <= 0 || H <= 0 || D <= 0) return -1;
+  if (p_e4m3 && !(p_lag >= 0.0 && std::isfinite(p_shift))) return -1;
   if (mode == 0 && !L_seq) return -1;
   if (mode == 1 && (n_cal <= 0 || !L_cal)) return -1;
   for (int i = 0; i < n_units; ++i) {
@@ -237,7 +284,7 @@ int oracle_walk(const uint16_t* q, const uint16_t* k, const uint16_t* v, const i
     const int S = cu_seqlens[sq + 1] - cu_seqlens[sq];
     if (qb * kTile >= S || (S + kTile - 1) / kTile > max_tiles) return -1;
   }
-  Problem P{q, k, v, cu_seqlens, batch, H, D, oracle_score_scale(softmax_scale, D)};
+  Problem P{q, k, v, cu_seqlens, batch, H, D, oracle_score_scale(softmax_scale, D), p_e4m3, p_shift, p_lag, out_scale};
   std::atomic<int> next{0};
   auto worker = [&]() {
     for (int i = next++; i < n_units; i = next++) {

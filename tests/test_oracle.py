@@ -326,3 +326,113 @@ def test_fit_and_resolve_reject_degenerate_input():
         oracle.fit_logspace([0.0, 1.0], [1.0, 2.0])
     assert math.isnan(oracle.resolve(-1.0, 2.0, 0.5))
     assert math.isnan(oracle.resolve(1.0, 2.0, 1.5))
+
+
+# ------------------------------------------------------ 8-bit P.V reading
+
+
+def e4m3_values():
+    """Every non-negative finite E4M3 value, built from the bit fields (4
+    exponent bits, bias 7, 3 mantissa bits, exponent field 0 subnormal, the
+    all-ones pattern S.1111.111 not a number)."""
+    vals = []
+    for e in range(16):
+        for m in range(8):
+            if e == 15 and m == 7:
+                continue
+            vals.append(m / 8 * 2.0 ** -6 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7))
+    return np.array(sorted(vals))
+
+
+def test_e4m3_nearest_is_the_brute_force_nearest_value():
+    """The oracle's rounding equals the nearest value of the enumerated E4M3
+    set, ties to the value with an even mantissa, saturating at 448; and it
+    agrees with the input quantiser's independent implementation."""
+    vals = e4m3_values()
+    assert len(vals) == 127 and vals[-1] == 448.0 and vals[1] == 2.0 ** -9
+    rng = np.random.default_rng(3)
+    xs = np.concatenate([vals, (vals[1:] + vals[:-1]) / 2,  # every midpoint: a tie
+                         rng.uniform(0, 460, 3000), np.exp2(rng.uniform(-14, 9, 3000)), [460.0, 1e6]])
+    codes = {v: i for i, v in enumerate(vals)}
+    for x in xs:
+        got = oracle.e4m3_nearest(float(x))
+        if x >= 448.0:
+            assert got == 448.0
+            continue
+        d = np.abs(vals - x)
+        best = vals[d == d.min()]
+        if len(best) == 2:  # tie: the even code (mantissa LSB 0) wins
+            best = [b for b in best if codes[b] % 2 == 0]
+        assert got == best[0], (x, got, best)
+    q = synth.f32_to_e4m3(np.asarray(xs[xs < 448], dtype=np.float32))
+    np.testing.assert_array_equal(synth.e4m3_to_f32(q).astype(np.float64),
+                                  [oracle.e4m3_nearest(float(np.float32(x))) for x in xs[xs < 448]])
+
+
+def _integer_score_case(S, D=16, seed=0, spread=5):
+    """Q, K with small integers so that every score q.k is an integer, and a
+    softmax scale whose log2-domain factor is exactly 1: s2 = q.k."""
+    rng = np.random.default_rng(seed)
+    q = np.zeros((S, 1, D), np.float32)
+    q[:, 0, :3] = rng.integers(0, 2, (S, 3))  # rows differ in which of three score terms they see
+    k = rng.integers(-1, 2, (S, 1, D)).astype(np.float32)
+    k[:, 0, :3] = rng.integers(0, spread, (S, 3))  # scores q.k in [0, 3 (spread - 1)]
+    v = rng.standard_normal((S, 1, D)).astype(np.float32)
+    scale = math.log(2.0)
+    assert oracle.score_scale(scale, D) == 1.0
+    return as_bf16(q), as_bf16(k), as_bf16(v), np.array([0, S], np.int32), scale
+
+
+def test_e4m3_pv_is_exact_when_every_probability_is_a_power_of_two():
+    """Integer scores (window of a few units): against the integer reference
+    every P = 2^(s - r + 8) is a power of two inside the E4M3 range, so the
+    8-bit P.V walk must give the exact walk's output; rescales are powers of
+    two as well. (A wrong reference or shift would push P out of range.)"""
+    q, k, v, cu, scale = _integer_score_case(300)
+    exact = oracle.walk(q, k, v, cu, 1, 16, softmax_scale=scale, tsf=0.0)
+    pv8 = oracle.walk(q, k, v, cu, 1, 16, softmax_scale=scale, tsf=0.0, p_e4m3=True)
+    np.testing.assert_allclose(pv8["out"], exact["out"], rtol=1e-6, atol=1e-7)
+    # a shift that would push P over 448 saturates, and then the outputs differ
+    sat = oracle.walk(q, k, v, cu, 1, 16, softmax_scale=scale, tsf=0.0, p_e4m3=True, p_shift=10.0)
+    assert np.abs(sat["out"] - exact["out"]).max() > 1e-3
+
+
+def test_e4m3_pv_single_tile_by_hand():
+    """One row, one tile: P_c = 2^(s_c - ceil(max s) + 8), O = sum(round(P_c) v_c) / sum(P_c)
+    with round() the brute-force nearest E4M3 value; V one-hot per column so
+    each output coordinate isolates one rounded probability."""
+    S, D = 9, 16
+    s = np.array([0.3, -1.7, 2.2, 2.45, -5.1, 0.0, 1.15, -0.6, 2.4])  # log2-domain scores
+    q = np.zeros((S, 1, D), np.float32)
+    k = np.zeros((S, 1, D), np.float32)
+    q[:, 0, 0] = 1.0
+    k[:, 0, 0] = s  # q.k = s for the first query row (other rows: same)
+    v = np.zeros((S, 1, D), np.float32)
+    for c in range(S):
+        v[c, 0, c] = 1.0
+    qb, kb, vb = as_bf16(q), as_bf16(k), as_bf16(v)
+    s_bf = synth.bf16_to_f32(kb[:, 0, 0]).astype(np.float64)  # the scores after bf16 rounding of k
+    res = oracle.walk(qb, kb, vb, np.array([0, S], np.int32), 1, D, softmax_scale=math.log(2.0), tsf=0.0,
+                      p_e4m3=True)
+    vals = e4m3_values()
+    r = math.ceil(s_bf.max())
+    P = 2.0 ** (s_bf - r + 8)
+    Pq = np.array([vals[np.argmin(np.abs(vals - p))] for p in P])  # no ties among these values
+    expect = Pq / P.sum()
+    np.testing.assert_allclose(res["out"][0, 0, :S], expect, rtol=1e-6)
+
+
+def test_e4m3_pv_error_bound_against_the_exact_walk():
+    """Rounding P to E4M3 moves each product by at most 2^-4 of it, and the
+    flushed values are below 2^-10 against a row maximum above 2^7, so
+    |O_8bit - O_exact| <= (2^-4 + S * 2^-17) * max|V| per row."""
+    w, q, k, v = varlen_random([1000, 333], 2, 64, seed=8)
+    cu = w.cu_seqlens
+    exact = oracle.walk(q, k, v, cu, 2, 64, tsf=0.0)
+    pv8 = oracle.walk(q, k, v, cu, 2, 64, tsf=0.0, p_e4m3=True)
+    vmax = np.abs(synth.bf16_to_f32(v)).max()
+    err = np.abs(pv8["out"] - exact["out"]).max()
+    assert err <= (2.0 ** -4 + 1000 * 2.0 ** -17) * vmax
+    assert err > 0  # the rounding is really applied
+    sk = oracle.walk(q, k, v, cu, 2, 64, tsf=500.0, p_e4m3=True)  # the skip rule does not change
+    assert np.array_equal(sk["decision"], oracle.walk(q, k, v, cu, 2, 64, tsf=500.0)["decision"])
