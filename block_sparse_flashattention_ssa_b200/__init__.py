@@ -9,7 +9,8 @@ fails loudly when the library is missing.
 Entry points (same names as the C ABI, without the ``ssa_`` prefix):
   fwd          skip-softmax attention forward (optionally with per-tile
                diagnostics, the ``ssa_fwd_ex`` call)
-  fwd_fp8      the forward with E4M3 Q and K (per-tensor descales)
+  fwd_fp8      the forward with E4M3 Q and K, or Q, K and V (per-tensor
+               descales; ssa_fwd_fp8 / ssa_fwd_fp8_qkv)
   quantize_fp8 bf16 -> E4M3 per-tensor quantisation for fwd_fp8
   calibrate    dense attention + skip counts at N thresholds at once
                (optionally with the per-tile statistic, ``ssa_calibrate_ex``)
@@ -62,6 +63,12 @@ def _load():
     L.ssa_calibrate_fp8.restype = i32
     L.ssa_calibrate_fp8.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32, vp, i32, vp, vp, i32,
                                     vp]
+    L.ssa_fwd_fp8_qkv.restype = i32
+    L.ssa_fwd_fp8_qkv.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32, f32, f32, vp, vp, i32,
+                                  vp, vp, vp]
+    L.ssa_calibrate_fp8_qkv.restype = i32
+    L.ssa_calibrate_fp8_qkv.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32, f32, f32, f32, f32, vp, i32, vp,
+                                        vp, i32, vp]
     L.ssa_quantize_fp8.restype = i32
     L.ssa_quantize_fp8.argtypes = [vp, vp, ctypes.c_int64, f32, vp]
     L.ssa_calibrate.restype = i32
@@ -142,7 +149,7 @@ def _require(t, name, dtype, device, shape=None, allow_none=False):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
-def _check_attention_args(q, k, v, cu_seqlens, out, qk_dtype):
+def _check_attention_args(q, k, v, cu_seqlens, out, qk_dtype, v_dtype=None):
     import torch
 
     if not (isinstance(q, torch.Tensor) and q.is_cuda):
@@ -151,7 +158,7 @@ def _check_attention_args(q, k, v, cu_seqlens, out, qk_dtype):
     shape = tuple(q.shape)
     _require(q, "q", qk_dtype, dev)
     _require(k, "k", qk_dtype, dev, shape)
-    _require(v, "v", torch.bfloat16, dev, shape)
+    _require(v, "v", v_dtype or torch.bfloat16, dev, shape)
     _require(cu_seqlens, "cu_seqlens", torch.int32, dev)
     if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
         raise ValueError("cu_seqlens must be a 1-D tensor of batch + 1 offsets")
@@ -224,23 +231,29 @@ def fwd(q, k, v, cu_seqlens, max_seqlen: int, threshold_scale_factor: float = 0.
 
 def fwd_fp8(q8, k8, v, cu_seqlens, max_seqlen: int, q_descale: float, k_descale: float,
             threshold_scale_factor: float = 0.0, softmax_scale: float = 0.0, out=None, skip_counter=None,
-            decision_bitmap=None, tile_stat=None, stream=None):
+            decision_bitmap=None, tile_stat=None, v_descale=None, stream=None):
     """Forward with E4M3 Q and K (CUDA uint8 [total_tokens, H, 128], values
-    q_descale * decode(q8)) and bf16 V; returns bf16 ``out``."""
+    q_descale * decode(q8)); returns bf16 ``out``. V is bf16 (ssa_fwd_fp8) or,
+    with ``v_descale``, E4M3 codes as well, P then rounded to E4M3 for the
+    P.V product (ssa_fwd_fp8_qkv)."""
     import torch
 
     total, H, D = _shape(q8)
-    dev = _check_attention_args(q8, k8, v, cu_seqlens, out, torch.uint8)
+    qkv = v_descale is not None
+    dev = _check_attention_args(q8, k8, v, cu_seqlens, out, torch.uint8, torch.uint8 if qkv else None)
     batch = cu_seqlens.numel() - 1
     nq = _per_unit_qblocks(dev, H, total, batch, _forward_outputs(skip_counter, decision_bitmap, tile_stat,
                                                                   max_seqlen))
     if out is None:
-        out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
-    rc = _lib.ssa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D,
-                          float(softmax_scale), float(q_descale), float(k_descale), float(threshold_scale_factor),
-                          _ptr(out), _ptr(skip_counter), nq, _ptr(decision_bitmap), _ptr(tile_stat),
-                          _stream_handle(stream))
-    _check(rc, "ssa_fwd_fp8")
+        out = torch.empty(v.shape, dtype=torch.bfloat16, device=v.device)
+    head = [_ptr(q8), _ptr(k8), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D,
+            float(softmax_scale), float(q_descale), float(k_descale)]
+    tail = [float(threshold_scale_factor), _ptr(out), _ptr(skip_counter), nq, _ptr(decision_bitmap),
+            _ptr(tile_stat), _stream_handle(stream)]
+    if qkv:
+        _check(_lib.ssa_fwd_fp8_qkv(*head, float(v_descale), *tail), "ssa_fwd_fp8_qkv")
+    else:
+        _check(_lib.ssa_fwd_fp8(*head, *tail), "ssa_fwd_fp8")
     return out
 
 
@@ -289,23 +302,28 @@ def calibrate(q, k, v, cu_seqlens, max_seqlen: int, thresholds, softmax_scale: f
 
 
 def calibrate_fp8(q8, k8, v, cu_seqlens, max_seqlen: int, q_descale: float, k_descale: float, thresholds,
-                  softmax_scale: float = 0.0, out=None, counts=None, stream=None):
-    """calibrate() on the E4M3 scores of fwd_fp8. Returns (out, counts[H, Q, N])."""
+                  softmax_scale: float = 0.0, out=None, counts=None, v_descale=None, stream=None):
+    """calibrate() on the E4M3 scores of fwd_fp8 (V bf16, or E4M3 codes with
+    ``v_descale``: ssa_calibrate_fp8_qkv). Returns (out, counts[H, Q, N])."""
     import torch
 
     total, H, D = _shape(q8)
-    dev = _check_attention_args(q8, k8, v, cu_seqlens, out, torch.uint8)
+    qkv = v_descale is not None
+    dev = _check_attention_args(q8, k8, v, cu_seqlens, out, torch.uint8, torch.uint8 if qkv else None)
     th = np.ascontiguousarray(thresholds, dtype=np.float32)
     batch = cu_seqlens.numel() - 1
     if counts is None:
         counts = torch.empty((H, num_qblocks(cu_seqlens), len(th)), dtype=torch.int32, device=dev)
     nq = _per_unit_qblocks(dev, H, total, batch, [(counts, "counts", torch.int32, (len(th),))])
     if out is None:
-        out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
-    rc = _lib.ssa_calibrate_fp8(_ptr(q8), _ptr(k8), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D,
-                                float(softmax_scale), float(q_descale), float(k_descale), th.ctypes.data, len(th),
-                                _ptr(out), _ptr(counts), nq, _stream_handle(stream))
-    _check(rc, "ssa_calibrate_fp8")
+        out = torch.empty(v.shape, dtype=torch.bfloat16, device=v.device)
+    head = [_ptr(q8), _ptr(k8), _ptr(v), _ptr(cu_seqlens), batch, total, int(max_seqlen), H, D,
+            float(softmax_scale), float(q_descale), float(k_descale)]
+    tail = [th.ctypes.data, len(th), _ptr(out), _ptr(counts), nq, _stream_handle(stream)]
+    if qkv:
+        _check(_lib.ssa_calibrate_fp8_qkv(*head, float(v_descale), *tail), "ssa_calibrate_fp8_qkv")
+    else:
+        _check(_lib.ssa_calibrate_fp8(*head, *tail), "ssa_calibrate_fp8")
     return out, counts
 
 

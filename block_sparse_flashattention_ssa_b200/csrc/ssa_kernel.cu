@@ -17,7 +17,8 @@
 //   warp 9  tcgen05 issuer, per KV tile j and per block X in order A, B:
 //           O_X += P_X V_j (when X keeps j, P_X read from TMEM), then
 //           S_X = Q_X K_{j+1}^T into the same TMEM columns (bf16 operands, or
-//           E4M3 ones with per-tensor descales folded into the score scale).
+//           E4M3 ones with per-tensor descales folded into the score scale;
+//           with E4M3 V the P V product runs on E4M3 P and V as well).
 // tcgen05 MMAs issued by one thread execute in issue order, so the S MMA
 // cannot overwrite P_X before the PV MMA ahead of it has read P_X; and a
 // commit tracks every earlier MMA of the thread, so when S_X(j+1) is reported
@@ -34,7 +35,8 @@
 // and calibration kernels to columns [0,64) in kv order, in the skipping
 // kernel kv [0,64) to columns [0,32) and kv [64,128) to [64,96), so the upper
 // half can be stored as soon as it is computed (its S columns have been read)
-// while the lower half of S is still being read back.
+// while the lower half of S is still being read back. E4M3 P (four kv per
+// column) goes to columns [0,16) and [64,80) in every kernel.
 //
 // Every wait on an mbarrier is bounded in time; when one runs out the CTA
 // records SSA_ERR_TIMEOUT in the device status word, the other roles see the
@@ -97,6 +99,7 @@ struct Params {
   int batch, total_tokens, num_heads, max_tiles, bitmap_words;
   int nq_check;  // q-blocks the per-unit outputs are sized for, or -1 when there are none
   float c;    // fp32(softmax_scale * log2 e)
+  float v_scale;  // multiplies the output: the V descale for E4M3 V, else 1
   float tsf;  // threshold_scale_factor (kSkip)
   int n_cal;
   float Lcal[SSA_MAX_THRESHOLDS];  // fp32(log2 lambda_k) (kCalib)
@@ -117,15 +120,22 @@ struct Ctl {
   int seq, qb_a, has_b, S, start, gqb_a, nq_total;
 };
 
-// Shared-memory layout. Q and K are bf16, or E4M3 bytes when F8; V is bf16.
-// Every tile is stored as chunks of 128 rows x 128 B with the 128-byte swizzle.
-template <int D, bool F8>
+// Operand precisions: bf16 everywhere; E4M3 Q and K; E4M3 Q, K, V and P.
+enum Prec : int { kBf16 = 0, kQK8 = 1, kQKV8 = 2 };
+
+// Shared-memory layout. Q and K are bf16, or E4M3 bytes from kQK8 on; V is
+// bf16, or E4M3 bytes for kQKV8. Every tile is stored as chunks of 128 rows x
+// 128 B with the 128-byte swizzle.
+template <int D, int PREC>
 struct Layout {
-  static constexpr int kQKElem = F8 ? 1 : 2;                  // bytes per Q/K element
+  static constexpr int kQKElem = PREC >= kQK8 ? 1 : 2;        // bytes per Q/K element
   static constexpr int kQKTileBytes = kBM * D * kQKElem;
   static constexpr int kQKChunkElems = 128 / kQKElem;         // Q/K elements per 128-B row of a chunk
   static constexpr int kQKChunks = D / kQKChunkElems;
-  static constexpr int kVTileBytes = kBN * D * 2;
+  static constexpr int kVElem = PREC == kQKV8 ? 1 : 2;        // bytes per V element
+  static constexpr int kVChunkElems = 128 / kVElem;           // V elements per 128-B row of a chunk
+  static constexpr int kVChunks = D / kVChunkElems;
+  static constexpr int kVTileBytes = kBN * D * kVElem;
   static constexpr int kChunkBytes = kBM * 128;
   static constexpr int kQ = 0;  // Q_A, then Q_B
   static constexpr int kK = kQ + kQBlocks * kQKTileBytes;
@@ -293,11 +303,13 @@ __device__ void locate_unit(const Params& p, bool need_max, int lane, Ctl& ctl) 
   }
 }
 
-template <int D, int MODE, bool EX, bool F8>
+template <int D, int MODE, bool EX, int PREC>
 __global__ void __launch_bounds__(kThreads, 1)
     ssa_attention_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params p) {
-  using L = Layout<D, F8>;
+  using L = Layout<D, PREC>;
+  constexpr bool F8 = PREC >= kQK8;    // S = Q K^T on E4M3 operands
+  constexpr bool F8V = PREC == kQKV8;  // O += P V on E4M3 operands as well
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl& ctl = *reinterpret_cast<Ctl*>(smem + L::kCtl);
@@ -404,8 +416,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t dst = smem_u32(smem + L::kV + vs * L::kVTileBytes);
           mbar_arrive_expect_tx(v_full(vs), L::kVTileBytes);
-          for (int ch = 0; ch < D / 64; ++ch)
-            tma_load_3d(dst + ch * L::kChunkBytes, &tmV, v_full(vs), ch * 64, head, seq_start + j * kBN);
+          for (int ch = 0; ch < L::kVChunks; ++ch)
+            tma_load_3d(dst + ch * L::kChunkBytes, &tmV, v_full(vs), ch * L::kVChunkElems, head,
+                        seq_start + j * kBN);
           ++v_issued;
         }
       }
@@ -421,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------- tcgen05 issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_f32(kBM, kBN) : idesc_bf16_f32(kBM, kBN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
+      constexpr uint32_t idesc_pv = F8V ? idesc_e4m3_f32(kBM, D, true) : idesc_bf16_f32(kBM, D, true);
       // S_X = Q_X K_t^T (the caller has made sure K_t has landed and that
       // nothing still needs S_X's previous contents).
       auto issue_qk = [&](int x, int t) {
@@ -443,17 +456,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(s_full(x));
       };
       // O_X += P_X V from the TMEM copy of P_X and V stage vs. The skipping
-      // kernel keeps P of kv [64,128) at columns [64,96) of S_X.
+      // kernel keeps bf16 P of kv [64,128) at columns [64,96) of S_X; E4M3 P
+      // (every kernel) sits at columns [0,16) and [64,80).
       auto issue_pv = [&](int x, int vs, bool accumulate) {
         const uint32_t p_tmem = tmem + col_S(x);
         const uint32_t v_s = smem_u32(smem + L::kV + vs * L::kVTileBytes);
+        if (F8V) {
+          // E4M3 P four to a column, 32 kv per instruction; V MN-major with
+          // its 128 E4M3 d values in one 128-B row per kv: 32 rows = 4 KB per
+          // k step, one swizzle atom across d (LBO unused), 8-row groups 1 KB
+          // apart.
 #pragma unroll
-        for (int ks = 0; ks < kBN / 16; ++ks) {
-          // V is MN-major (d contiguous): 16 kv rows = 2 KB per k step; the
-          // second 64-column chunk of d sits one 16 KB chunk further (LBO).
-          const uint32_t p_col = ks * 8 + ((MODE == kSkip && ks >= kBN / 32) ? 32 : 0);
-          mma_ts(tmem + col_O(x), p_tmem + p_col, smem_desc_sw128(v_s + ks * 16 * 128, L::kChunkBytes, 1024),
-                 idesc_pv, (accumulate || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < kBN / 32; ++ks) {
+            const uint32_t p_col = ks * 8 + (ks >= kBN / 64 ? 48 : 0);
+            mma_ts_f8(tmem + col_O(x), p_tmem + p_col, smem_desc_sw128(v_s + ks * 32 * 128, 0, 1024), idesc_pv,
+                      (accumulate || ks > 0) ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < kBN / 16; ++ks) {
+            // V is MN-major (d contiguous): 16 kv rows = 2 KB per k step; the
+            // second 64-column chunk of d sits one 16 KB chunk further (LBO).
+            const uint32_t p_col = ks * 8 + ((MODE == kSkip && ks >= kBN / 32) ? 32 : 0);
+            mma_ts(tmem + col_O(x), p_tmem + p_col, smem_desc_sw128(v_s + ks * 16 * 128, L::kChunkBytes, 1024),
+                   idesc_pv, (accumulate || ks > 0) ? 1u : 0u);
+          }
         }
       };
       bool ok = wait_bar(bar_q, 0, abort_flag) && wait_bar(k_full(0), 0, abort_flag);
@@ -619,9 +646,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_new = fmaxf(m_true, tmax);
       m_true = m_new;
       float alpha = 1.f;
-      if (__any_sync(kFull, m_new > m_used + kRescaleThreshold)) {
-        alpha = ex2_approx(m_used - m_new);  // 0 before the first kept tile
-        m_used = m_new;
+      // Reference of the exponentials. bf16 P: m_used, moved to m_true only
+      // once m_true passes it by kRescaleThreshold, so O is rescaled rarely.
+      // E4M3 P: an integer r >= m_true (held in m_used), raised to
+      // ceil(m_true) as soon as m_true passes it, so that P = 2^(s2 - r + 8)
+      // lies in (0, 256], inside E4M3's range, and every rescale factor
+      // 2^(r_old - r_new) is an exact power of two.
+      const bool up = F8V ? m_new > m_used : m_new > m_used + kRescaleThreshold;
+      if (__any_sync(kFull, up)) {
+        if (F8V) {
+          if (up) {
+            const float r_new = ceilf(m_new);
+            const float e = m_used - r_new;  // a negative integer, or -inf before the first kept tile
+            alpha = e < -126.f ? 0.f : __int_as_float((static_cast<int>(e) + 127) << 23);
+            m_used = r_new;
+          }
+        } else {
+          alpha = ex2_approx(m_used - m_new);  // 0 before the first kept tile
+          m_used = m_new;
+        }
         if (kept > 0) {
 #pragma unroll
           for (int ch = 0; ch < D / 32; ++ch) {
@@ -634,41 +677,79 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       l *= alpha;
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_used, -m_used);
+      const float bias = F8V ? 8.f - m_used : -m_used;
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(bias, bias);
       float2 rs[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       uint32_t lo[64];
       tmem_ld_x64_async(lane_base + col_s, lo);  // lands while the upper half is exponentiated
-      // Packed P: bf16 pairs of consecutive kv columns. The dense and
-      // calibration kernels keep all 64 pairs in registers and store them to
-      // columns [0,64) at once; the skipping kernel, which has less register
-      // room, stores the upper half's pairs to columns [64,96) right away.
-      uint32_t pk[64];
+      if (F8V) {
+        // E4M3 P, four consecutive kv per column: kv [64,128) stored to
+        // columns [64,80) as soon as computed (those S columns have been
+        // read), kv [0,64) to columns [0,16) once the lower half is back.
+        uint32_t pk[16];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float2 a = ffma2(make_float2(__uint_as_float(hi[2 * i]), __uint_as_float(hi[2 * i + 1])), c2, nm2);
-        const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
-        rs[i & 1] = fadd2(rs[i & 1], e);
-        pk[32 + i] = pack_bf16x2(e.x, e.y);
-      }
-      if (MODE == kSkip) tmem_st_x32(lane_base + col_s + 64, reinterpret_cast<const uint32_t(&)[32]>(pk[32]));
-      tmem_wait_ld_tied(lo);
-      if (valid < 64) {
+        for (int i = 0; i < 16; ++i) {
+          const float2 a0 = ffma2(make_float2(__uint_as_float(hi[4 * i]), __uint_as_float(hi[4 * i + 1])), c2, nm2);
+          const float2 a1 =
+              ffma2(make_float2(__uint_as_float(hi[4 * i + 2]), __uint_as_float(hi[4 * i + 3])), c2, nm2);
+          const float2 e0 = make_float2(ex2_approx(a0.x), ex2_approx(a0.y));
+          const float2 e1 = make_float2(ex2_approx(a1.x), ex2_approx(a1.y));
+          rs[0] = fadd2(rs[0], e0);
+          rs[1] = fadd2(rs[1], e1);
+          pk[i] = pack_e4m3x2(e0.x, e0.y) | (pack_e4m3x2(e1.x, e1.y) << 16);
+        }
+        tmem_st_x16(lane_base + col_s + 64, pk);
+        tmem_wait_ld_tied(lo);
+        if (valid < 64) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i)
-          if (i >= valid) lo[i] = __float_as_uint(-INFINITY);
-      }
+          for (int i = 0; i < 64; ++i)
+            if (i >= valid) lo[i] = __float_as_uint(-INFINITY);
+        }
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float2 a = ffma2(make_float2(__uint_as_float(lo[2 * i]), __uint_as_float(lo[2 * i + 1])), c2, nm2);
-        const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
-        rs[i & 1] = fadd2(rs[i & 1], e);
-        pk[i] = pack_bf16x2(e.x, e.y);
+        for (int i = 0; i < 16; ++i) {
+          const float2 a0 = ffma2(make_float2(__uint_as_float(lo[4 * i]), __uint_as_float(lo[4 * i + 1])), c2, nm2);
+          const float2 a1 =
+              ffma2(make_float2(__uint_as_float(lo[4 * i + 2]), __uint_as_float(lo[4 * i + 3])), c2, nm2);
+          const float2 e0 = make_float2(ex2_approx(a0.x), ex2_approx(a0.y));
+          const float2 e1 = make_float2(ex2_approx(a1.x), ex2_approx(a1.y));
+          rs[0] = fadd2(rs[0], e0);
+          rs[1] = fadd2(rs[1], e1);
+          pk[i] = pack_e4m3x2(e0.x, e0.y) | (pack_e4m3x2(e1.x, e1.y) << 16);
+        }
+        tmem_st_x16(lane_base + col_s, pk);
+      } else {
+        // Packed P: bf16 pairs of consecutive kv columns. The dense and
+        // calibration kernels keep all 64 pairs in registers and store them to
+        // columns [0,64) at once; the skipping kernel, which has less register
+        // room, stores the upper half's pairs to columns [64,96) right away.
+        uint32_t pk[64];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float2 a = ffma2(make_float2(__uint_as_float(hi[2 * i]), __uint_as_float(hi[2 * i + 1])), c2, nm2);
+          const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+          rs[i & 1] = fadd2(rs[i & 1], e);
+          pk[32 + i] = pack_bf16x2(e.x, e.y);
+        }
+        if (MODE == kSkip) tmem_st_x32(lane_base + col_s + 64, reinterpret_cast<const uint32_t(&)[32]>(pk[32]));
+        tmem_wait_ld_tied(lo);
+        if (valid < 64) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            if (i >= valid) lo[i] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float2 a = ffma2(make_float2(__uint_as_float(lo[2 * i]), __uint_as_float(lo[2 * i + 1])), c2, nm2);
+          const float2 e = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+          rs[i & 1] = fadd2(rs[i & 1], e);
+          pk[i] = pack_bf16x2(e.x, e.y);
+        }
+        // Both halves of S_X are in registers by now: P_X may overwrite them.
+        if (MODE == kSkip)
+          tmem_st_x32(lane_base + col_s, reinterpret_cast<const uint32_t(&)[32]>(pk[0]));
+        else
+          tmem_st_x64(lane_base + col_s, pk);
       }
-      // Both halves of S_X are in registers by now: P_X may overwrite them.
-      if (MODE == kSkip)
-        tmem_st_x32(lane_base + col_s, reinterpret_cast<const uint32_t(&)[32]>(pk[0]));
-      else
-        tmem_st_x64(lane_base + col_s, pk);
       l += (rs[0].x + rs[1].x) + (rs[0].y + rs[1].y);
       warp_arrive(p_ready(x), lane);
       ++kept;
@@ -683,7 +764,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) ok = warp_wait(o_final, 0, abort_flag);
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.0f / l;
+      const float inv_l = F8V ? p.v_scale / l : 1.0f / l;
       __nv_bfloat16* orow =
           p.out + (static_cast<int64_t>(seq_start + qb * kBM + row) * p.num_heads + head) * static_cast<int64_t>(D);
 #pragma unroll
@@ -782,7 +863,9 @@ struct Call {
   void* out;
   cudaStream_t stream;
   bool f8 = false;              // Q and K are E4M3 bytes
+  bool f8v = false;             // V is E4M3 bytes too (and P is rounded to E4M3)
   double qk_descale = 1.0;      // q_descale * k_descale (E4M3 only)
+  float v_descale = 1.0f;       // multiplies the output when V is E4M3
 };
 
 // True when `p` is device (or managed) memory of the current device: a host
@@ -816,6 +899,7 @@ int validate(const Call& a) {
   if (a.D != 64 && a.D != 128) return SSA_ERR_UNSUPPORTED;
   if (a.f8 && a.D != 128) return SSA_ERR_UNSUPPORTED;  // E4M3 rows of 128 B: one swizzle atom per row
   if (a.f8 && !(a.qk_descale > 0.0 && std::isfinite(a.qk_descale))) return SSA_ERR_INVALID_ARG;
+  if (a.f8v && !(a.v_descale > 0.f && std::isfinite(a.v_descale))) return SSA_ERR_INVALID_ARG;
   if (a.total_tokens == 0) return SSA_OK;
   if (!a.q || !a.k || !a.v || !a.out) return SSA_ERR_INVALID_ARG;
   for (const void* ptr : {a.q, a.k, a.v, static_cast<const void*>(a.out)})
@@ -836,19 +920,21 @@ Params base_params(const Call& a) {
   double scale = a.softmax_scale > 0.f ? static_cast<double>(a.softmax_scale) : 1.0 / std::sqrt(static_cast<double>(a.D));
   if (a.f8) scale = scale * a.qk_descale;  // E4M3 codes carry the per-tensor scales of Q and K
   p.c = static_cast<float>(scale * 1.4426950408889634073599246810019);
+  p.v_scale = a.f8v ? a.v_descale : 1.0f;
   return p;
 }
 
-template <int D, int MODE, bool EX, bool F8>
+template <int D, int MODE, bool EX, int PREC>
 int launch(const Call& a, const Params& p) {
   CUtensorMap tq, tk, tv;
-  if (!make_tensor_map(&tq, a.q, a.total_tokens, a.H, D, F8) || !make_tensor_map(&tk, a.k, a.total_tokens, a.H, D, F8) ||
-      !make_tensor_map(&tv, a.v, a.total_tokens, a.H, D, false)) {
+  if (!make_tensor_map(&tq, a.q, a.total_tokens, a.H, D, PREC >= kQK8) ||
+      !make_tensor_map(&tk, a.k, a.total_tokens, a.H, D, PREC >= kQK8) ||
+      !make_tensor_map(&tv, a.v, a.total_tokens, a.H, D, PREC == kQKV8)) {
     t_last_cuda_error = "cuTensorMapEncodeTiled failed or the driver entry point is unavailable";
     return SSA_ERR_CUDA;
   }
-  auto kernel = ssa_attention_kernel<D, MODE, EX, F8>;
-  constexpr int smem = Layout<D, F8>::kAlloc;
+  auto kernel = ssa_attention_kernel<D, MODE, EX, PREC>;
+  constexpr int smem = Layout<D, PREC>::kAlloc;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e);
   // one CTA per pair of query blocks: sum over sequences of ceil(S_b / 256) <= ceil(T / 256) + batch
@@ -861,8 +947,9 @@ int launch(const Call& a, const Params& p) {
 
 template <int MODE, bool EX>
 int dispatch_d(const Call& a, const Params& p) {
-  if (a.f8) return launch<128, MODE, EX, true>(a, p);
-  return a.D == 64 ? launch<64, MODE, EX, false>(a, p) : launch<128, MODE, EX, false>(a, p);
+  if (a.f8v) return launch<128, MODE, EX, kQKV8>(a, p);
+  if (a.f8) return launch<128, MODE, EX, kQK8>(a, p);
+  return a.D == 64 ? launch<64, MODE, EX, kBf16>(a, p) : launch<128, MODE, EX, kBf16>(a, p);
 }
 
 // y = E4M3(fp32(x * inv_scale)), round to nearest even, saturating to +-448;
@@ -932,6 +1019,21 @@ extern "C" int ssa_fwd_fp8(const void* q, const void* k, const void* v, const in
     return SSA_ERR_INVALID_ARG;
   a.f8 = true;
   a.qk_descale = static_cast<double>(q_descale) * static_cast<double>(k_descale);
+  return fwd_impl(a, threshold_scale_factor, skip_counter, num_qblocks, decision_bitmap, tile_stat);
+}
+
+extern "C" int ssa_fwd_fp8_qkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                               int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                               float q_descale, float k_descale, float v_descale, float threshold_scale_factor,
+                               void* out, int32_t* skip_counter, int num_qblocks, uint32_t* decision_bitmap,
+                               float* tile_stat, void* stream) {
+  Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
+         static_cast<cudaStream_t>(stream)};
+  if (!(q_descale > 0.f) || !(k_descale > 0.f) || std::isinf(q_descale) || std::isinf(k_descale))
+    return SSA_ERR_INVALID_ARG;
+  a.f8 = a.f8v = true;
+  a.qk_descale = static_cast<double>(q_descale) * static_cast<double>(k_descale);
+  a.v_descale = v_descale;
   return fwd_impl(a, threshold_scale_factor, skip_counter, num_qblocks, decision_bitmap, tile_stat);
 }
 
@@ -1021,6 +1123,21 @@ extern "C" int ssa_calibrate_fp8(const void* q, const void* k, const void* v, co
     return SSA_ERR_INVALID_ARG;
   a.f8 = true;
   a.qk_descale = static_cast<double>(q_descale) * static_cast<double>(k_descale);
+  return calibrate_impl(a, thresholds, n_thresholds, counts, num_qblocks, nullptr);
+}
+
+extern "C" int ssa_calibrate_fp8_qkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens,
+                                     int batch, int total_tokens, int max_seqlen, int num_heads, int head_dim,
+                                     float softmax_scale, float q_descale, float k_descale, float v_descale,
+                                     const float* thresholds, int n_thresholds, void* out, int32_t* counts,
+                                     int num_qblocks, void* stream) {
+  Call a{q, k, v, cu_seqlens, batch, total_tokens, max_seqlen, num_heads, head_dim, softmax_scale, out,
+         static_cast<cudaStream_t>(stream)};
+  if (!(q_descale > 0.f) || !(k_descale > 0.f) || std::isinf(q_descale) || std::isinf(k_descale))
+    return SSA_ERR_INVALID_ARG;
+  a.f8 = a.f8v = true;
+  a.qk_descale = static_cast<double>(q_descale) * static_cast<double>(k_descale);
+  a.v_descale = v_descale;
   return calibrate_impl(a, thresholds, n_thresholds, counts, num_qblocks, nullptr);
 }
 

@@ -167,6 +167,40 @@ int ssa_fwd_fp8(const void* q, const void* k, const void* v, const int32_t* cu_s
                 uint32_t* decision_bitmap, float* tile_stat, void* stream);
 
 /*
+ * ssa_fwd_fp8 with V in E4M3 as well, and P rounded to E4M3 for the P.V
+ * product: both MMAs run on 8-bit operands (tcgen05 kind::f8f6f4). The
+ * TRT-LLM pull-request page ("Benchmark") reports skip-softmax speed-ups with
+ * FP8 and NVFP4 attention; the docs ("User Configuration") name skip-softmax
+ * combined with quantised attention. Reading, where the pages are silent:
+ * one scale per tensor (real V = v_descale * decode(v)); the skip rule and
+ * its running max m are those of ssa_fwd; each row takes its probabilities
+ * against an integer reference r >= m that moves to ceil(m) as soon as m
+ * passes it (rescaling O and l by the exact power of two 2^(r_old - r_new)),
+ * P = 2^(s2 - r + 8) in (0, 256], the P.V product uses P rounded to the
+ * nearest E4M3 value while the row sum l adds the unrounded P, and the output
+ * is v_descale * O / l in bf16.
+ *   q, k, v     device E4M3 bytes [total_tokens, num_heads, 128]
+ *   out         device bf16 [total_tokens, num_heads, 128]
+ *   q_descale, k_descale, v_descale  > 0, finite
+ *   other arguments as in ssa_fwd_fp8
+ */
+int ssa_fwd_fp8_qkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                    int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                    float q_descale, float k_descale, float v_descale, float threshold_scale_factor, void* out,
+                    int32_t* skip_counter, int num_qblocks, uint32_t* decision_bitmap, float* tile_stat,
+                    void* stream);
+
+/*
+ * ssa_calibrate with E4M3 Q, K and V: the dense pass of ssa_fwd_fp8_qkv and its
+ * counts (which depend on Q and K only, so they equal ssa_calibrate_fp8's).
+ * Arguments as in ssa_calibrate_fp8, plus v_descale.
+ */
+int ssa_calibrate_fp8_qkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens, int batch,
+                          int total_tokens, int max_seqlen, int num_heads, int head_dim, float softmax_scale,
+                          float q_descale, float k_descale, float v_descale, const float* thresholds,
+                          int n_thresholds, void* out, int32_t* counts, int num_qblocks, void* stream);
+
+/*
  * Per-tensor E4M3 quantisation for ssa_fwd_fp8: y[i] = E4M3(fp32(x[i] * inv_scale)),
  * round to nearest even, saturating to +-448 (a caller with amax = max|x|
  * passes inv_scale = 448 / amax and then q_descale = 1 / inv_scale).

@@ -131,6 +131,17 @@ def test_fp8_entry_points_validate_on_the_host(ssa):
     assert f8(q=mis) == ssa.SSA_ERR_UNSUPPORTED
     assert f8(tsf=float("nan")) == ssa.SSA_ERR_INVALID_ARG
     assert f8(total=0) == ssa.SSA_OK
+    def f8v(vd=1.0, D=128, total=256):
+        return L.ssa_fwd_fp8_qkv(fake, fake, fake, fake, 1, total, 256, 2, D, 0.0, 1.0, 1.0, vd, 0.0, fake, None, 0,
+                                 None, None, None)
+
+    assert f8v(vd=0.0) == ssa.SSA_ERR_INVALID_ARG
+    assert f8v(vd=float("inf")) == ssa.SSA_ERR_INVALID_ARG
+    assert f8v(D=64) == ssa.SSA_ERR_UNSUPPORTED
+    assert f8v(total=0) == ssa.SSA_OK
+    th = np.array([1e-3], dtype=np.float32)
+    assert L.ssa_calibrate_fp8_qkv(fake, fake, fake, fake, 1, 256, 256, 2, 128, 0.0, 1.0, 1.0, -1.0, th.ctypes.data,
+                                   1, fake, fake, 2, None) == ssa.SSA_ERR_INVALID_ARG
     qz = lambda x, y, n, s: L.ssa_quantize_fp8(x, y, n, s, None)
     assert qz(fake, fake, -1, 1.0) == ssa.SSA_ERR_INVALID_ARG
     assert qz(fake, fake, 16, 0.0) == ssa.SSA_ERR_INVALID_ARG

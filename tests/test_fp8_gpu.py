@@ -143,3 +143,74 @@ def test_fp8_wan14b_at_the_benchmarked_threshold(ssa):
     _check(case, 0.0, units=units, what="wan14b fp8 dense")
     _, skip = _check(case, tsf, units=units, what="wan14b fp8 target 0.7")
     assert skip.sum() > 0
+
+
+class Fp8QkvCase(Case):
+    """Q, K and V quantised per tensor on the GPU (ssa_fwd_fp8_qkv): the
+    oracle walks the exactly decoded values with the Q/K descales in its
+    softmax scale, the 8-bit P.V reading (P rounded to E4M3 against the
+    per-row integer reference) and the V descale on its output."""
+
+    def __init__(self, ssa, w):
+        q, k, v = synth.generate(w)
+        self.q8, self.q_inv, self.q_ds = synth.quantize_e4m3(q)
+        self.k8, self.k_inv, self.k_ds = synth.quantize_e4m3(k)
+        self.v8, self.v_inv, self.v_ds = synth.quantize_e4m3(v)
+        dec = lambda c: synth.f32_to_bf16(synth.e4m3_to_f32(c))
+        super().__init__(ssa, w, dec(self.q8), dec(self.k8), dec(self.v8))
+        self.dq8 = _device_codes(ssa, q, self.q_inv)
+        self.dk8 = _device_codes(ssa, k, self.k_inv)
+        self.dv8 = _device_codes(ssa, v, self.v_inv)
+        torch.cuda.synchronize()
+        for dev_codes, host_codes in ((self.dq8, self.q8), (self.dk8, self.k8), (self.dv8, self.v8)):
+            assert np.array_equal(dev_codes.cpu().numpy(), host_codes)
+        self.oracle_scale = 1.0 / math.sqrt(w.D) * (float(self.q_ds) * float(self.k_ds))
+        self.oracle_kw = dict(p_e4m3=True, out_scale=float(self.v_ds))
+
+    def call(self, tsf, out, skip, bitmap, stat):
+        self.ssa.fwd_fp8(self.dq8, self.dk8, self.dv8, self.dcu, self.w.max_seqlen, float(self.q_ds),
+                         float(self.k_ds), tsf, out=out, skip_counter=skip, decision_bitmap=bitmap, tile_stat=stat,
+                         v_descale=float(self.v_ds))
+
+
+def test_fp8_qkv_ragged_varlen(ssa):
+    """E4M3 Q, K, V and P on ragged lengths (1 .. 1000, an empty sequence),
+    dense and lambda below and above 1: outputs, decisions, statistics and
+    skip counts against the oracle; the call without diagnostics equals the
+    diagnostic one bit for bit."""
+    lengths = [1, 5, 127, 128, 129, 300, 0, 1000]
+    w = synth.Workload("ragged fp8 qkv", [(1, 1, s) for s in lengths], H=3, D=128, seed=12, amp=3.0)
+    case = Fp8QkvCase(ssa, w)
+    for tsf in [0.0, 50.0, 300.0, 2000.0]:
+        _check(case, tsf, what="ragged fp8 qkv")
+
+
+def test_fp8_qkv_wan5b_sampled(ssa):
+    case = Fp8QkvCase(ssa, synth.WAN5B)
+    units = oracle.sample_units(case.cu, case.w.H, 24, seed=4)
+    for tsf in [0.0, 5e3, 2e4]:
+        _check(case, tsf, units=units, what="wan5b fp8 qkv")
+
+
+def test_fp8_qkv_calibration(ssa):
+    """ssa_calibrate_fp8_qkv: its output is the dense E4M3 Q/K/V output (the
+    oracle's dense walk with the 8-bit P.V reading, and ssa_fwd_fp8_qkv at
+    tsf = 0 bit for bit); its counts depend on Q and K only, so they equal
+    ssa_calibrate_fp8's on the same E4M3 Q and K."""
+    lams = synth.CALIB_THRESHOLDS
+    w = synth.Workload("calib fp8 qkv", [(1, 1, 300), (1, 1, 129), (1, 1, 1000)], H=2, D=128, seed=13, amp=3.0)
+    case = Fp8QkvCase(ssa, w)
+    out, counts = ssa.calibrate_fp8(case.dq8, case.dk8, case.dv8, case.dcu, w.max_seqlen, float(case.q_ds),
+                                    float(case.k_ds), lams, v_descale=float(case.v_ds))
+    ssa.check_device()
+    v_bf16 = torch.from_numpy(synth.generate(w)[2].view(np.int16)).cuda().view(torch.bfloat16)
+    _, counts_qk = ssa.calibrate_fp8(case.dq8, case.dk8, v_bf16, case.dcu, w.max_seqlen, float(case.q_ds),
+                                     float(case.k_ds), lams)
+    ssa.check_device()
+    assert torch.equal(counts, counts_qk)
+    res = case.walk(cal_lambdas=lams)
+    st = parity.Stats()
+    parity.compare_calibration(res, case.cu, [oracle.lambda_log2(x) for x in lams], parity.bf16_host(out),
+                               counts.cpu().numpy(), st, what="calib fp8 qkv")
+    st.check("calib fp8 qkv")
+    np.testing.assert_array_equal(parity.bf16_host(out), case.fwd(0.0, ex=False)[0])

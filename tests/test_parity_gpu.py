@@ -34,6 +34,7 @@ class Case:
     """Host inputs, their device copies and the GPU runs of one workload."""
 
     oracle_scale = 0.0  # softmax_scale the oracle is given (0: 1/sqrt(D))
+    oracle_kw = {}      # further oracle arguments of the variant (the 8-bit P.V reading)
 
     def __init__(self, ssa, w: synth.Workload, q=None, k=None, v=None):
         self.ssa, self.w = ssa, w
@@ -64,7 +65,7 @@ class Case:
 
     def walk(self, **kw):
         return oracle.walk(self.q, self.k, self.v, self.cu, self.w.H, self.w.D, softmax_scale=self.oracle_scale,
-                           max_tiles=self.T, **kw)
+                           max_tiles=self.T, **self.oracle_kw, **kw)
 
     def L_seq(self, tsf):
         return [oracle.threshold_log2(tsf, s) for s in self.w.seqlens]
