@@ -10,7 +10,11 @@ batch, at the threshold_scale_factor resolved for target sparsity 0.7 from an
 a*exp(b*s) model that ssa_calibrate + ssa_fit_logspace fit on this same input
 before timing (calibrate at the deployment shape; the fit is done once, the
 target resolved on the host). The dense run (tsf = 0, the same kernel with
-skipping off) and the other targets (0.5, 0.9) are timed beside it.
+skipping off) and the other targets (0.5, 0.9) are timed beside it, with the
+E4M3 variants (Q/K, and Q/K/V) at dense and the target-0.7 threshold, and the
+other specified workloads (the pages' example formula on the same input, the
+S = 8192 threshold sweep, the 4-sequence varlen batch): none of them is in
+the timed region.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 Prints one JSON line on rank 0.
@@ -66,19 +70,22 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(workload: str, tsf: float):
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def measured_traffic(workload: str, tsf: float, path: str = TRAFFIC_FILE):
     """DRAM bytes per launch (read + write) from a committed ncu capture of
-    this exact kernel source, workload and threshold; None otherwise."""
-    path = os.path.join(ROOT, "profiles", "ssa_attention_wan14b_dram.md")
+    this exact kernel source, workload and threshold (profiles/traffic.json:
+    a list of {"hash", "workload", "tsf", "bytes"} records); None otherwise."""
     if not os.path.exists(path):
         return None
     want = kernel_source_hash()
-    for line in open(path):
-        if not line.startswith("traffic:"):
-            continue
-        kv = dict(x.split("=", 1) for x in line.split()[1:])
-        if kv.get("hash") == want and kv.get("workload") == workload and abs(float(kv["tsf"]) - tsf) <= 1e-6 * max(1.0, tsf):
-            return float(kv["bytes"])
+    with open(path) as f:
+        records = json.load(f)
+    for r in records:
+        if r.get("hash") == want and r.get("workload") == workload and \
+                abs(float(r["tsf"]) - tsf) <= 1e-6 * max(1.0, tsf):
+            return float(r["bytes"])
     return None
 
 
@@ -215,6 +222,80 @@ def time_fwd(ssa, args_fn, reps, stream):
     return [e0.elapsed_time(e1) for e0, e1 in evs]
 
 
+def device_inputs(w, dev):
+    """Seeded host Q/K/V of workload w and their device copies."""
+    import torch
+
+    import synth
+
+    q, k, v = synth.generate(w)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    return (q, k, v), (to_dev(q), to_dev(k), to_dev(v), torch.from_numpy(w.cu_seqlens).to(dev))
+
+
+def threshold_rows(ssa, w, dq, dk, dv, dcu, tsfs, reps, stream, names=None):
+    """Median CUDA-event time, skip ratio and throughput of ssa_fwd at each
+    threshold_scale_factor (three untimed calls first); speedups are over
+    the first entry, which is tsf = 0 (the same kernel with skipping off)."""
+    import torch
+
+    skip = torch.zeros((w.H, ssa.num_qblocks(w.cu_seqlens)), dtype=torch.int32, device=dq.device)
+    out = torch.empty_like(dq)
+    tiles = tiles_of(w.seqlens, w.H)
+    rows = []
+    for i, t in enumerate(tsfs):
+        call = lambda t=t: ssa.fwd(dq, dk, dv, dcu, w.max_seqlen, t, out=out, skip_counter=skip)
+        for _ in range(3):
+            call()
+        ms = statistics.median(time_fwd(ssa, call, reps, stream))
+        ssa.check_device()
+        r = float(skip.sum().item()) / tiles
+        row = dict(tsf=t, ms=ms, skip_ratio=r, dense_eq_tflops=w.dense_flop() / ms / 1e9,
+                   effective_tflops=algorithmic_flop(w.seqlens, w.D, w.H, r) / ms / 1e9)
+        if names is not None:
+            row["name"] = names[i]
+        rows.append(row)
+    for r in rows:
+        r["speedup_vs_dense"] = rows[0]["ms"] / r["ms"]
+        if r["skip_ratio"] > 0:
+            r["f"] = (1.0 - r["ms"] / rows[0]["ms"]) / r["skip_ratio"]
+    return rows
+
+
+def specified_workloads(ssa, stream, dev, main_inputs, reps=5):
+    """The other workloads the benchmark is specified on, timed beside the
+    headline (not in its timed region): the S = 75,600 input at the pages'
+    example formula a = 0.0003, b = 7.5 (s = 0.5 / 0.7 / 0.9); the WAN-5B-like
+    S = 8192 sweep; the 4-sequence varlen batch at tsf = 5000 and at the
+    target-0.7 threshold of its own per-sequence calibration fit."""
+    import torch
+
+    import synth
+    from block_sparse_flashattention_ssa_b200 import calibration as cal
+
+    out = {}
+    w14 = synth.WAN14B
+    dq, dk, dv, dcu = main_inputs
+    out["wan14b_page_formula"] = threshold_rows(
+        ssa, w14, dq, dk, dv, dcu, SWEEPS["wan14b"], reps, stream,
+        names=["dense"] + [f"page_formula_{s}" for s in TARGETS])
+    w5 = synth.WAN5B
+    _, (q5, k5, v5, cu5) = device_inputs(w5, dev)
+    out["wan5b_sweep"] = threshold_rows(ssa, w5, q5, k5, v5, cu5, SWEEPS["wan5b"], 20, stream)
+    del q5, k5, v5
+    wv = synth.VARLEN
+    _, (qv, kv, vv, cuv) = device_inputs(wv, dev)
+    c = cal.calibrate(qv, kv, vv, cuv, wv.max_seqlen)
+    ssa.check_device()
+    tsf07 = ssa.resolve(c.a, c.b, HEADLINE_TARGET)
+    out["varlen"] = threshold_rows(ssa, wv, qv, kv, vv, cuv, [0.0, 5000.0, tsf07], reps, stream,
+                                   names=["dense", "tsf_5000", f"fitted_target_{HEADLINE_TARGET}"])
+    out["varlen_fit"] = {"a": c.a, "b": c.b, "s_min": c.s_min, "s_max": c.s_max}
+    del qv, kv, vv
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
 
@@ -259,28 +340,38 @@ def run_ours(args):
         r = float(skip.sum().item()) / tiles
         rows[name] = dict(tsf=t, ms=ms, skip_ratio=r, dense_eq_tflops=dense_flop / ms / 1e9,
                           effective_tflops=algorithmic_flop(w.seqlens, w.D, w.H, r) / ms / 1e9)
-    # side rows of the E4M3 Q/K variant (ssa_fwd_fp8) at the same thresholds
+    # side rows of the E4M3 variants at the same thresholds: Q and K
+    # (ssa_fwd_fp8), and Q, K, V with E4M3 P (ssa_fwd_fp8_qkv)
     if fit is not None and w.D == 128:
         _, q_inv, q_ds = synth.quantize_e4m3(q)
         _, k_inv, k_ds = synth.quantize_e4m3(k)
+        _, v_inv, v_ds = synth.quantize_e4m3(v)
         dq8, dk8 = ssa.quantize_fp8(dq, float(q_inv)), ssa.quantize_fp8(dk, float(k_inv))
-        step8 = lambda t: ssa.fwd_fp8(dq8, dk8, dv, dcu, w.max_seqlen, float(q_ds), float(k_ds), t, out=out,
-                                      skip_counter=skip)
-        for name, t in [("fp8_qk_dense", 0.0), (f"fp8_qk_target_{HEADLINE_TARGET}", tsf)]:
-            for _ in range(2):
-                step8(t)
-            ms = statistics.median(time_fwd(ssa, lambda: step8(t), 5, stream))
-            ssa.check_device()
-            r = float(skip.sum().item()) / tiles
-            rows[name] = dict(tsf=t, ms=ms, skip_ratio=r, dense_eq_tflops=dense_flop / ms / 1e9,
-                              qk_dtype="e4m3 (per-tensor descale)")
-        del dq8, dk8
+        dv8 = ssa.quantize_fp8(dv, float(v_inv))
+        variants = {"fp8_qk": (lambda t: ssa.fwd_fp8(dq8, dk8, dv, dcu, w.max_seqlen, float(q_ds), float(k_ds), t,
+                                                     out=out, skip_counter=skip), "e4m3 Q, K (per-tensor descale)"),
+                    "fp8_qkv": (lambda t: ssa.fwd_fp8(dq8, dk8, dv8, dcu, w.max_seqlen, float(q_ds), float(k_ds), t,
+                                                      out=out, skip_counter=skip, v_descale=float(v_ds)),
+                                "e4m3 Q, K, V and P (per-tensor descales)")}
+        for prefix, (step8, what) in variants.items():
+            for name, t in [(f"{prefix}_dense", 0.0), (f"{prefix}_target_{HEADLINE_TARGET}", tsf)]:
+                for _ in range(2):
+                    step8(t)
+                ms = statistics.median(time_fwd(ssa, lambda: step8(t), 5, stream))
+                ssa.check_device()
+                r = float(skip.sum().item()) / tiles
+                rows[name] = dict(tsf=t, ms=ms, skip_ratio=r, dense_eq_tflops=dense_flop / ms / 1e9, operands=what)
+        del dq8, dk8, dv8
     dense_ms = rows["dense"]["ms"] if "dense" in rows else None
     for name, r in rows.items() if dense_ms else []:
-        base = rows["fp8_qk_dense"]["ms"] if name.startswith("fp8") else dense_ms  # same-precision dense
+        prefix = "fp8_qkv" if name.startswith("fp8_qkv") else "fp8_qk" if name.startswith("fp8_qk") else None
+        base = rows[prefix + "_dense"]["ms"] if prefix else dense_ms  # the dense run of the same precision
         r["speedup_vs_dense"] = base / r["ms"]
         if r["skip_ratio"] > 0:
             r["f"] = (1.0 - r["ms"] / base) / r["skip_ratio"]
+    specified = None
+    if fit is not None and args.workload == "wan14b" and not args.no_side_workloads:
+        specified = specified_workloads(ssa, stream, dev, (dq, dk, dv, dcu))
 
     # timed region
     for _ in range(args.warmup):
@@ -351,6 +442,7 @@ def run_ours(args):
         "dense_ms": dense_ms,
         "fit": fit,
         "targets": rows,
+        "specified_workloads": specified,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": p_burst, "unit": "TFLOP/s",
                      "frac": achieved / p_burst, "traffic": measured_traffic(args.workload, tsf),
                      "peak_kind": f"{peak_kind} bf16 burst", "peak_sustained": p_sus,
@@ -417,7 +509,7 @@ def cpu_baseline(w, q, k, v, budget_s=12.0, tsf=None):
     dt = time.time() - t0
     flop = 4.0 * rows * S * w.D
     return {"value": flop / dt / 1e12, "unit": "TFLOP/s (dense-equivalent)", "cores": cores, "kind": "oracle",
-            "sample": f"{done} (head, q-block) units of the S=75,600 workload ({rows} query rows, "
+            "sample": f"{done} (head, q-block) units of the {w.name} workload ({rows} query rows, "
                       f"{dt:.1f} s wall), tsf={tsf or 0.0:.6g}"}
 
 
@@ -428,7 +520,7 @@ def run_reference(args):
         return
     import synth
 
-    w = synth.WAN14B
+    w = getattr(synth, WORKLOADS[args.workload])
     q, k, v = synth.generate(w)
     for _ in range(args.warmup):
         pass  # the oracle has no warm-up state; warm-up steps are free
@@ -529,32 +621,40 @@ def run_tsf_sweep(args):
 
     dev = torch.device("cuda", 0)
     w = getattr(synth, WORKLOADS[args.workload])
-    q, k, v = synth.generate(w)
-    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
-    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
-    dcu = torch.from_numpy(w.cu_seqlens).to(dev)
-    skip = torch.zeros((w.H, ssa.num_qblocks(w.cu_seqlens)), dtype=torch.int32, device=dev)
-    out = torch.empty_like(dq)
-    stream = torch.cuda.current_stream()
-    tiles = tiles_of(w.seqlens, w.H)
+    _, (dq, dk, dv, dcu) = device_inputs(w, dev)
     reps = 5 if w.dense_flop() > 1e14 else 20
-    rows = []
-    for t in SWEEPS[args.workload]:
-        call = lambda t=t: ssa.fwd(dq, dk, dv, dcu, w.max_seqlen, t, out=out, skip_counter=skip)
-        for _ in range(3):
-            call()
-        ms = statistics.median(time_fwd(ssa, call, reps, stream))
-        ssa.check_device()
-        r = float(skip.sum().item()) / tiles
-        rows.append(dict(tsf=t, ms=ms, skip_ratio=r, dense_eq_tflops=w.dense_flop() / ms / 1e9,
-                         effective_tflops=algorithmic_flop(w.seqlens, w.D, w.H, r) / ms / 1e9))
-    for r in rows:
-        r["speedup_vs_dense"] = rows[0]["ms"] / r["ms"]
+    rows = threshold_rows(ssa, w, dq, dk, dv, dcu, SWEEPS[args.workload], reps, torch.cuda.current_stream())
     qkv = 3 * w.total_tokens * w.H * w.D * 2
     print(json.dumps({"metric": "skip-softmax forward at the specified thresholds",
                       "config": {"workload": w.name, "reps": reps, "qkv_bytes": qkv,
                                  "l2": "inputs larger than L2" if qkv > 126e6 else "inputs fit in L2"},
                       "rows": rows}), flush=True)
+
+
+def ensure_world(gpus: int) -> None:
+    """Make the process layout match --gpus N: under torchrun the world size
+    must equal N (otherwise exit 2); a plain `python bench.py --gpus N` with
+    N > 1 re-executes itself under torch.distributed.run with N local ranks
+    on 127.0.0.1 and exits with its status."""
+    world = int(os.environ.get("WORLD_SIZE", "0"))
+    if world:
+        if world != gpus:
+            print(f"bench.py: --gpus {gpus} but WORLD_SIZE={world}", file=sys.stderr)
+            sys.exit(2)
+        return
+    if gpus == 1:
+        return
+    if gpus < 1:
+        print(f"bench.py: --gpus {gpus} must be >= 1", file=sys.stderr)
+        sys.exit(2)
+    import socket
+
+    with socket.socket() as sk:  # a free port for the rendezvous
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    sys.exit(subprocess.call(cmd))
 
 
 def main():
@@ -565,6 +665,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-side-workloads", action="store_true",
+                    help="skip the side rows of the other specified workloads (page formula, S=8192 sweep, varlen)")
     ap.add_argument("--workload", default="wan14b", choices=sorted(WORKLOADS),
                     help="problem shape (the default is the benchmark workload; the others serve profiling)")
     ap.add_argument("--calib-sweep", action="store_true",
@@ -574,6 +676,7 @@ def main():
     ap.add_argument("--tsf", type=float, default=None,
                     help="fixed threshold_scale_factor: skip calibration and the side rows")
     args = ap.parse_args()
+    ensure_world(args.gpus)
     if args.impl == "reference":
         run_reference(args)
     elif args.calib_sweep:
