@@ -25,9 +25,12 @@
 // complete every MMA into O_X issued before it has completed too (the softmax
 // may rescale O_X and overwrite the P_X columns without a further wait).
 // A block's skip decision reaches the issuer as a tagged word in shared
-// memory that it polls with acquire loads (the producer, which decides the V
-// loads, waits on a barrier instead): on the issuing thread a barrier wait
-// stalls longer behind its in-flight MMAs than a load does.
+// memory that it polls with acquire loads (on the issuing thread a barrier
+// wait stalls longer behind its in-flight MMAs than a load does); the
+// producer, which decides the V loads, polls the same word with a back-off.
+// In the skipping kernel the decision also says that K_{j+1} has landed (the
+// group's first warp waits for it before it reads S_X(j)), so the issuer puts
+// S_X(j+1) in flight with no wait of its own.
 // The two softmax groups run out of phase: one group's exponentials overlap
 // the MMAs of the other.
 // TMEM (512 columns): S_A [0,128) S_B [128,256) O_A [256,256+D)
@@ -110,7 +113,6 @@ struct Ctl {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[kQBlocks], p_ready[kQBlocks];
-  uint64_t dec_ready[kQBlocks][kDecRing];
   uint64_t o_final, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -173,6 +175,27 @@ __device__ __forceinline__ bool wait_decision(uint32_t addr, int tag, int& word,
     word = ld_acquire_shared(addr);
     if ((word >> 1) == tag) return true;
     if ((i & 31u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicOr(&g_status, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// Same, for a waiter that is in no hurry: sleeps between polls, so that it
+// leaves shared-memory bandwidth to the tensor cores' operand reads.
+__device__ __forceinline__ bool wait_decision_sleep(uint32_t addr, int tag, int& word, volatile int* abort_flag) {
+  word = ld_acquire_shared(addr);
+  if ((word >> 1) == tag) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(64);
+    word = ld_acquire_shared(addr);
+    if ((word >> 1) == tag) return true;
+    if ((i & 15u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
         *abort_flag = 1;
@@ -333,7 +356,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto v_empty = [&](int i) { return smem_u32(&ctl.v_empty[i]); };
   auto s_full = [&](int x) { return smem_u32(&ctl.s_full[x]); };
   auto p_ready = [&](int x) { return smem_u32(&ctl.p_ready[x]); };
-  auto dec_ready = [&](int x, int i) { return smem_u32(&ctl.dec_ready[x][i]); };
   const uint32_t o_final = smem_u32(&ctl.o_final);
 
   if (threadIdx.x == 0) {
@@ -349,7 +371,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < kQBlocks; ++x) {
       mbar_init(s_full(x), 1);
       mbar_init(p_ready(x), 4);  // one arrival per softmax warp of the group, per kept tile
-      for (int i = 0; i < kDecRing; ++i) mbar_init(dec_ready(x, i), 1);
     }
     mbar_init(o_final, 1);
     mbar_init(smem_u32(&ctl.drain), 1);
@@ -400,11 +421,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (MODE == kSkip) {  // V_j is needed when either block keeps tile j
           need_v = false;
           for (int x = 0; x < nx && !need_v; ++x) {
-            if (!wait_bar(dec_ready(x, j % kDecRing), (j / kDecRing) & 1, abort_flag)) {
+            int word;
+            if (!wait_decision_sleep(smem_u32(&ctl.dec[x][j % kDecRing]), j + 1, word, abort_flag)) {
               ok = false;
               break;
             }
-            need_v = (reinterpret_cast<volatile int*>(ctl.dec[x])[j % kDecRing] & 1) == 0;
+            need_v = (word & 1) == 0;
           }
           if (!ok) break;
         }
@@ -493,10 +515,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       int v_used = 0;
       for (int j = 0; ok && j < nkv; ++j) {
         const int t = j + 1;  // S_X(t) is issued right behind O_X += P_X(j) V_j
-        // Waits that are normally already satisfied (K_{j+1}; in the dense and
-        // calibration orders also V_j) come first, while no MMA of this tile
-        // is in flight: a wait behind in-flight MMAs stalls the issuer.
-        if (t < nkv && !(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag))) break;
+        // Waits that are normally already satisfied (K_{j+1} and V_j in the
+        // dense and calibration orders) come first, while no MMA of this tile
+        // is in flight: a wait behind in-flight MMAs stalls the issuer. In the
+        // skipping order the decisions polled below imply K_{j+1}.
+        if (MODE != kSkip && t < nkv && !(ok = wait_bar(k_full(t % kKStages), (t / kKStages) & 1, abort_flag)))
+          break;
         bool v_waited = false;
         if (MODE != kSkip) {
           if (!(ok = wait_bar(v_full(v_used % kVStages), (v_used / kVStages) & 1, abort_flag))) break;
@@ -505,7 +529,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int x = 0; x < nx; ++x) {
           bool skip = false;
           if (MODE == kSkip) {
-            // The decision also says every warp of the group has read S_X(j).
+            // The decision also says every warp of the group has read S_X(j)
+            // and that K_{j+1} has landed.
             int word;
             if (!(ok = wait_decision(smem_u32(&ctl.dec[x][j % kDecRing]), j + 1, word, abort_flag))) break;
             skip = (word & 1) != 0;
@@ -565,6 +590,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
 
     for (int j = 0; j < nkv; ++j) {
+      // Skipping order: the group's first warp (which publishes the decision)
+      // makes sure K_{j+1} has landed, while it would wait for S_X(j) anyway.
+      if (MODE == kSkip && wq == 0 && j + 1 < nkv &&
+          !(ok = warp_wait(k_full((j + 1) % kKStages), ((j + 1) / kKStages) & 1, abort_flag)))
+        break;
       if (!(ok = warp_wait(s_full(x), j & 1, abort_flag))) break;
       tc_fence_after();
       // S_X is read whole for the row max; only its upper 64 columns stay in
@@ -633,7 +663,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (MODE == kSkip && gt == 0) {
           st_release_shared(smem_u32(&ctl.dec[x][j % kDecRing]), ((j + 1) << 1) | (skip ? 1 : 0));
-          mbar_arrive(dec_ready(x, j % kDecRing));
         }
       }
       if (skip) {  // nothing to hand over: P-ready counts kept tiles only
