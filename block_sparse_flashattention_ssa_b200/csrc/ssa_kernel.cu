@@ -34,12 +34,12 @@
 // The two softmax groups run out of phase: one group's exponentials overlap
 // the MMAs of the other.
 // TMEM (512 columns): S_A [0,128) S_B [128,256) O_A [256,256+D)
-// O_B [384,384+D); P_X is written over S_X as packed bf16 pairs: in the dense
-// and calibration kernels to columns [0,64) in kv order, in the skipping
-// kernel kv [0,64) to columns [0,32) and kv [64,128) to [64,96), so the upper
-// half can be stored as soon as it is computed (its S columns have been read)
-// while the lower half of S is still being read back. E4M3 P (four kv per
-// column) goes to columns [0,16) and [64,80) in every kernel.
+// O_B [384,384+D); P_X is written over S_X as packed bf16 pairs, kv [0,64) to
+// columns [0,32) and kv [64,128) to [64,96) (E4M3 P, four kv per column, to
+// [0,16) and [64,80)): the upper half is stored as soon as it is computed
+// (its S columns have been read) while the lower half of S is still being
+// read back, and the issuer starts O_X += P_X V on that half while the softmax
+// exponentiates the other one.
 //
 // Every wait on an mbarrier is bounded in time; when one runs out the CTA
 // records SSA_ERR_TIMEOUT in the device status word, the other roles see the
@@ -112,7 +112,7 @@ struct Ctl {
   uint64_t bar_q;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[kQBlocks], p_ready[kQBlocks];
+  uint64_t s_full[kQBlocks], p_hi[kQBlocks], p_ready[kQBlocks];
   uint64_t o_final, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -356,6 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto v_empty = [&](int i) { return smem_u32(&ctl.v_empty[i]); };
   auto s_full = [&](int x) { return smem_u32(&ctl.s_full[x]); };
   auto p_ready = [&](int x) { return smem_u32(&ctl.p_ready[x]); };
+  auto p_hi = [&](int x) { return smem_u32(&ctl.p_hi[x]); };
   const uint32_t o_final = smem_u32(&ctl.o_final);
 
   if (threadIdx.x == 0) {
@@ -371,6 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int x = 0; x < kQBlocks; ++x) {
       mbar_init(s_full(x), 1);
       mbar_init(p_ready(x), 4);  // one arrival per softmax warp of the group, per kept tile
+      mbar_init(p_hi(x), 4);     // the same, once the upper half of P_X is stored
     }
     mbar_init(o_final, 1);
     mbar_init(smem_u32(&ctl.drain), 1);
@@ -477,10 +479,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(s_full(x));
       };
-      // O_X += P_X V from the TMEM copy of P_X and V stage vs. The skipping
-      // kernel keeps bf16 P of kv [64,128) at columns [64,96) of S_X; E4M3 P
-      // (every kernel) sits at columns [0,16) and [64,80).
-      auto issue_pv = [&](int x, int vs, bool accumulate) {
+      // Half `half` of O_X += P_X V_vs from the TMEM copy of P_X: half 1 (kv
+      // [64,128)) is issued as soon as that half of P_X is stored, while the
+      // softmax still exponentiates the lower half; half 0 (kv [0,64)) once
+      // all of P_X is in place. P_X sits at columns [0,32) and [64,96) of S_X
+      // as bf16 pairs, or at [0,16) and [64,80) as E4M3.
+      auto issue_pv = [&](int x, int vs, int half, bool accumulate) {
         const uint32_t p_tmem = tmem + col_S(x);
         const uint32_t v_s = smem_u32(smem + L::kV + vs * L::kVTileBytes);
         if (F8V) {
@@ -489,19 +493,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           // k step, one swizzle atom across d (LBO unused), 8-row groups 1 KB
           // apart.
 #pragma unroll
-          for (int ks = 0; ks < kBN / 32; ++ks) {
-            const uint32_t p_col = ks * 8 + (ks >= kBN / 64 ? 48 : 0);
+          for (int i = 0; i < kBN / 64; ++i) {
+            const int ks = half * (kBN / 64) + i;
+            const uint32_t p_col = ks * 8 + (half ? 48 : 0);
             mma_ts_f8(tmem + col_O(x), p_tmem + p_col, smem_desc_sw128(v_s + ks * 32 * 128, 0, 1024), idesc_pv,
-                      (accumulate || ks > 0) ? 1u : 0u);
+                      (accumulate || i > 0) ? 1u : 0u);
           }
         } else {
 #pragma unroll
-          for (int ks = 0; ks < kBN / 16; ++ks) {
+          for (int i = 0; i < kBN / 32; ++i) {
             // V is MN-major (d contiguous): 16 kv rows = 2 KB per k step; the
             // second 64-column chunk of d sits one 16 KB chunk further (LBO).
-            const uint32_t p_col = ks * 8 + ((MODE == kSkip && ks >= kBN / 32) ? 32 : 0);
+            const int ks = half * (kBN / 32) + i;
+            const uint32_t p_col = ks * 8 + (half ? 32 : 0);
             mma_ts(tmem + col_O(x), p_tmem + p_col, smem_desc_sw128(v_s + ks * 16 * 128, L::kChunkBytes, 1024),
-                   idesc_pv, (accumulate || ks > 0) ? 1u : 0u);
+                   idesc_pv, (accumulate || i > 0) ? 1u : 0u);
           }
         }
       };
@@ -536,13 +542,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             skip = (word & 1) != 0;
           }
           if (!skip) {
-            if (!(ok = wait_bar(p_ready(x), kept[x] & 1, abort_flag))) break;
+            if (!(ok = wait_bar(p_hi(x), kept[x] & 1, abort_flag))) break;
             if (!v_waited) {
               if (!(ok = wait_bar(v_full(v_used % kVStages), (v_used / kVStages) & 1, abort_flag))) break;
               v_waited = true;
             }
             tc_fence_after();
-            issue_pv(x, v_used % kVStages, kept[x] > 0);
+            issue_pv(x, v_used % kVStages, 1, kept[x] > 0);
+            if (!(ok = wait_bar(p_ready(x), kept[x] & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_pv(x, v_used % kVStages, 0, true);
             ++kept[x];
           }
           if (t < nkv) {
@@ -728,6 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[i] = pack_e4m3x2(e0.x, e0.y) | (pack_e4m3x2(e1.x, e1.y) << 16);
         }
         tmem_st_x16(lane_base + col_s + 64, pk);
+        warp_arrive(p_hi(x), lane);
         tmem_wait_ld_tied(lo);
         if (valid < 64) {
 #pragma unroll
@@ -747,10 +757,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st_x16(lane_base + col_s, pk);
       } else {
-        // Packed P: bf16 pairs of consecutive kv columns. The dense and
-        // calibration kernels keep all 64 pairs in registers and store them to
-        // columns [0,64) at once; the skipping kernel, which has less register
-        // room, stores the upper half's pairs to columns [64,96) right away.
+        // Packed P: bf16 pairs of consecutive kv columns; the upper half's
+        // pairs go to columns [64,96) right away (the issuer starts on them),
+        // the lower half's to [0,32) once they are computed.
         uint32_t pk[64];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -759,7 +768,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           rs[i & 1] = fadd2(rs[i & 1], e);
           pk[32 + i] = pack_bf16x2(e.x, e.y);
         }
-        if (MODE == kSkip) tmem_st_x32(lane_base + col_s + 64, reinterpret_cast<const uint32_t(&)[32]>(pk[32]));
+        tmem_st_x32(lane_base + col_s + 64, reinterpret_cast<const uint32_t(&)[32]>(pk[32]));
+        warp_arrive(p_hi(x), lane);
         tmem_wait_ld_tied(lo);
         if (valid < 64) {
 #pragma unroll
@@ -774,10 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[i] = pack_bf16x2(e.x, e.y);
         }
         // Both halves of S_X are in registers by now: P_X may overwrite them.
-        if (MODE == kSkip)
-          tmem_st_x32(lane_base + col_s, reinterpret_cast<const uint32_t(&)[32]>(pk[0]));
-        else
-          tmem_st_x64(lane_base + col_s, pk);
+        tmem_st_x32(lane_base + col_s, reinterpret_cast<const uint32_t(&)[32]>(pk[0]));
       }
       l += (rs[0].x + rs[1].x) + (rs[0].y + rs[1].y);
       warp_arrive(p_ready(x), lane);

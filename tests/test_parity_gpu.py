@@ -174,11 +174,11 @@ def test_varlen_batch(ssa):
     check_forward(case, 5000.0, units=units, what="varlen", plain=True)
 
 
-def check_calibration(case, units=None, what=""):
+def check_calibration(case, units=None, what="", lams=None):
     """ssa_calibrate_ex (counts and every tile's statistic) against the
     oracle's calibration walk, tile by tile; plain ssa_calibrate must give
     the same output and counts bit for bit."""
-    lams = synth.CALIB_THRESHOLDS
+    lams = synth.CALIB_THRESHOLDS if lams is None else lams
     stat = torch.full((case.w.H, case.Q, case.T), float("nan"), dtype=torch.float32, device="cuda")
     out, counts = case.ssa.calibrate(case.dq, case.dk, case.dv, case.dcu, case.w.max_seqlen, lams, tile_stat=stat)
     case.ssa.check_device()
@@ -223,6 +223,25 @@ def test_calibration_varlen_sampled(ssa):
     case = Case(ssa, synth.VARLEN)
     units = oracle.sample_units(case.cu, case.w.H, 16, seed=5)
     check_calibration(case, units=units, what="calib varlen")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_more_than_32_sequences(ssa, D):
+    """A packed batch of 40 ragged sequences (empty, single-token, partial
+    and multi-tile ones): past 32 sequences the kernels map their CTAs to
+    (sequence, q-block pairs) in sequence order instead of longest first.
+    Forward at three thresholds and a calibration with the largest number of
+    trials one call takes (32), every unit against the oracle."""
+    rng = np.random.default_rng(40 + D)
+    lengths = [int(x) for x in rng.integers(0, 420, size=40)]
+    lengths[3], lengths[17], lengths[29] = 0, 1, 128
+    w = synth.Workload("40 sequences", [(1, 1, s) for s in lengths], H=2, D=D, seed=17, amp=3.0)
+    case = Case(ssa, w)
+    assert len(w.seqlens) > 32
+    for tsf in [0.0, 60.0, 400.0]:
+        check_forward(case, tsf, what=f"40 seqs D={D}", plain=True)
+    lams = [float(x) for x in np.geomspace(1e-6, 8.0, ssa.MAX_THRESHOLDS)]
+    check_calibration(case, what=f"calib 40 seqs D={D}", lams=lams)
 
 
 def test_d64_long_sequence_sampled(ssa):
