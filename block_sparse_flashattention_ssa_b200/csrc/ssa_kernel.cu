@@ -467,15 +467,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t d_tmem = tmem + col_S(x);
         // Shared-memory addresses stay below 256 KB, so the 14-bit address
         // field of a descriptor takes an offset by plain addition: each MMA's
-        // descriptors are the tile's plus a constant.
+        // descriptors are the tile's plus a constant, added to the low word
+        // alone (it cannot carry out of the field), which keeps the single
+        // issuing thread, on the critical path of every tile, short.
         const uint64_t da0 = smem_desc_sw128(q_s, 16, 1024), db0 = smem_desc_sw128(k_s, 16, 1024);
+        const uint32_t a_lo = static_cast<uint32_t>(da0), b_lo = static_cast<uint32_t>(db0);
+        const uint64_t a_hi = da0 & 0xFFFFFFFF00000000ull, b_hi = db0 & 0xFFFFFFFF00000000ull;
 #pragma unroll
         for (int ks = 0; ks < D * L::kQKElem / 32; ++ks) {
           // K-major, 128B swizzle: each MMA takes 32 B of K (16 bf16 or 32
           // E4M3 elements), 32 B apart inside a 128-B row; every 128 B of a
           // row start a new 16 KB chunk.
           const uint32_t off = (ks >> 2) * L::kChunkBytes + (ks & 3) * 32;
-          const uint64_t da = da0 + (off >> 4), db = db0 + (off >> 4);
+          const uint64_t da = a_hi | (a_lo + (off >> 4)), db = b_hi | (b_lo + (off >> 4));
           if (F8)
             mma_ss_f8(d_tmem, da, db, idesc_qk, ks > 0 ? 1u : 0u);
           else
@@ -497,23 +501,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           // k step, one swizzle atom across d (LBO unused), 8-row groups 1 KB
           // apart.
           const uint64_t vd0 = smem_desc_sw128(v_s, 0, 1024);
+          const uint32_t v_lo = static_cast<uint32_t>(vd0);
+          const uint64_t v_hi = vd0 & 0xFFFFFFFF00000000ull;
 #pragma unroll
           for (int i = 0; i < kBN / 64; ++i) {
             const int ks = half * (kBN / 64) + i;
             const uint32_t p_col = ks * 8 + (half ? 48 : 0);
-            mma_ts_f8(tmem + col_O(x), p_tmem + p_col, vd0 + static_cast<uint32_t>(ks * 32 * 128 >> 4), idesc_pv,
-                      (accumulate || i > 0) ? 1u : 0u);
+            mma_ts_f8(tmem + col_O(x), p_tmem + p_col, v_hi | (v_lo + static_cast<uint32_t>(ks * 32 * 128 >> 4)),
+                      idesc_pv, (accumulate || i > 0) ? 1u : 0u);
           }
         } else {
           // V is MN-major (d contiguous): 16 kv rows = 2 KB per k step; the
           // second 64-column chunk of d sits one 16 KB chunk further (LBO).
           const uint64_t vd0 = smem_desc_sw128(v_s, L::kChunkBytes, 1024);
+          const uint32_t v_lo = static_cast<uint32_t>(vd0);
+          const uint64_t v_hi = vd0 & 0xFFFFFFFF00000000ull;
 #pragma unroll
           for (int i = 0; i < kBN / 32; ++i) {
             const int ks = half * (kBN / 32) + i;
             const uint32_t p_col = ks * 8 + (half ? 32 : 0);
-            mma_ts(tmem + col_O(x), p_tmem + p_col, vd0 + static_cast<uint32_t>(ks * 16 * 128 >> 4), idesc_pv,
-                   (accumulate || i > 0) ? 1u : 0u);
+            mma_ts(tmem + col_O(x), p_tmem + p_col, v_hi | (v_lo + static_cast<uint32_t>(ks * 16 * 128 >> 4)),
+                   idesc_pv, (accumulate || i > 0) ? 1u : 0u);
           }
         }
       };
@@ -561,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++kept[x];
           }
           if (t < nkv) {
-            tc_fence_after();
+            if (skip) tc_fence_after();  // after a PV the fence above already covers the S MMAs
             issue_qk(x, t);
           }
         }
