@@ -21,7 +21,6 @@ information and the C fit drops them.
 """
 from __future__ import annotations
 
-import math
 import warnings
 from dataclasses import dataclass, field
 from typing import Callable, List, Optional, Sequence

@@ -20,7 +20,6 @@ import math
 
 import numpy as np
 
-import oracle
 import synth
 
 TILE = 128

@@ -6,8 +6,6 @@ Small cases are compared whole; the long-sequence workloads (S = 8192 and
 units that always holds q-block 0 and the tail q-block of every sequence:
 each unit's decisions and output rows depend on nothing outside it.
 """
-import math
-
 import numpy as np
 import pytest
 

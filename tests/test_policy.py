@@ -8,7 +8,6 @@ import math
 import numpy as np
 import pytest
 
-import block_sparse_flashattention_ssa_b200 as ssa
 from block_sparse_flashattention_ssa_b200.policy import DENSE, SKIP, GraphedAttention, SkipSoftmaxPolicy, dense_steps
 
 from tests import golden
